@@ -1,0 +1,162 @@
+"""Plant plausible mistakes in the oracle (CPU only) and require that a pin catches each.
+
+This shows the pins in test_oracle_pins.py are sensitive: a dropped term, a wrong sign,
+an off-by-one in the DCA remap, the mask or the selection each fails at least one check.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import dca_vs as O
+from tests import oracle_checks as C
+
+
+def _all_checks():
+    """name -> True when the check passes."""
+    res = {}
+    res["yarn"] = C.check_yarn_golden() < 1e-12
+    res["rope_tf"] = C.check_rope_vs_transformers() < 2e-4
+    res["rope_cplx"] = C.check_rope_complex() < 1e-12
+    res["dca_brute"] = C.check_dca_brute_force() < 1e-10
+    res["dca_inv"] = C.check_dca_invariants()
+    res["short"] = C.check_short_equals_causal_rope() < 1e-10
+    res["v_ones"] = C.check_v_ones() < 1e-12
+    res["full_budget"] = C.check_full_budget_is_dense() < 1e-12
+    res["est_mass"] = C.check_estimator_mass() < 1e-5
+    res["est_brute"] = C.check_estimator_brute_force() < 1e-6
+    res["topk"] = C.check_topk_properties()
+    res["force"] = C.check_force_local()
+    res["mask"] = C.check_mask_brute_force()
+    res["attended"] = C.check_attended_set()
+    return res
+
+
+def _rope_sign(x, pos, base):
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * O.rope_theta(d, base)
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., : d // 2], x[..., d // 2:]
+    return np.concatenate([x1 * c + x2 * s, x2 * c - x1 * s], axis=-1)
+
+
+def _rope_interleaved(x, pos, base):
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * O.rope_theta(d, base)
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = x1 * c - x2 * s
+    out[..., 1::2] = x2 * c + x1 * s
+    return out
+
+
+def _theta_wrong(d, base):
+    f = np.arange(d // 2, dtype=np.float64)
+    return np.power(float(base), -f / d)
+
+
+def _len_is_c(cfg):
+    return cfg.dca_chunk
+
+
+def _succ_clamp_c(i, pattern, cfg):
+    L, c = O.dca_len(cfg), cfg.dca_chunk
+    t = np.asarray(i) % L
+    if pattern == O.INTRA:
+        return t
+    if pattern == O.SUCC:
+        return np.minimum(t + L, c)
+    return np.full_like(t, c - 1)
+
+
+def _inter_at_c(i, pattern, cfg):
+    L, c = O.dca_len(cfg), cfg.dca_chunk
+    t = np.asarray(i) % L
+    if pattern == O.INTRA:
+        return t
+    if pattern == O.SUCC:
+        return np.minimum(t + L, c - 1)
+    return np.full_like(t, c)
+
+
+def _yarn_unsquared(s):
+    return 1.0 if s <= 1.0 else 0.1 * math.log(s) + 1.0
+
+
+def _scale_no_sqrt_d(cfg):
+    return O.yarn_inv_t(cfg.yarn_s)
+
+
+def _estimate_slash_unreversed(q_R, R, krot_g, e, cfg):
+    js = np.arange(e)
+    l = O.dca_logits(q_R, R, krot_g[:e], js, cfg)
+    l = np.where(js[None, :] <= R[:, None], l, -np.inf)
+    p, lse = O.softmax_rows(l)
+    slash = np.zeros(e)
+    for r, i in enumerate(R):
+        slash[: i + 1] += p[r, : i + 1]
+    return np.sum(p, 0).astype(np.float32), slash.astype(np.float32), lse
+
+
+def _estimator_rows_off(s0, e, cfg):
+    return np.arange(max(s0, e - cfg.vs_last_q - 1), e - 1)
+
+
+def _blocks_off_by_one(S, b, e, bs=O.BLOCK):
+    nkb = (e + bs - 1) // bs
+    r0, r1 = b * bs, min(b * bs + bs - 1, e - 1)
+    o = np.asarray(S, dtype=np.int64)
+    o = o[o <= r1]
+    lo, hi = np.maximum(0, r0 - o) // bs, (r1 - o) // bs
+    m = np.zeros(nkb, dtype=bool)
+    for a, z in zip(lo, hi):
+        m[a: z] = True          # drops the last block of each range
+    return m
+
+
+def _top_ties_reversed(scores, budget):
+    scores = np.asarray(scores, dtype=np.float64)
+    n = scores.shape[0]
+    if budget >= n:
+        return np.arange(n)
+    order = np.lexsort((-np.arange(n), -scores))
+    return np.sort(order[:budget])
+
+
+def _select_no_force(vert, slash, cfg):
+    return O.top_budget(vert, cfg.vs_vertical), O.top_budget(slash, cfg.vs_slash)
+
+
+def _attended_without_verticals(i, blocks, V, bs=O.BLOCK):
+    js = np.arange(i + 1)
+    return blocks[js // bs].copy()
+
+
+MUTATIONS = [
+    ("rope sign flipped", "rope", _rope_sign),
+    ("rope pairs interleaved", "rope", _rope_interleaved),
+    ("rope frequency exponent halved", "rope_theta", _theta_wrong),
+    ("DCA chunk length c instead of c - w", "dca_len", _len_is_c),
+    ("successive query clamped at c", "dca_query_position", _succ_clamp_c),
+    ("inter query at c", "dca_query_position", _inter_at_c),
+    ("YaRN factor not squared", "yarn_inv_t", _yarn_unsquared),
+    ("logit scale without 1/sqrt(D)", "logit_scale", _scale_no_sqrt_d),
+    ("slash offsets not reversed", "estimate_head", _estimate_slash_unreversed),
+    ("estimator rows shifted by one", "estimator_rows", _estimator_rows_off),
+    ("mask drops the last block of a slash range", "computed_blocks", _blocks_off_by_one),
+    ("top-k ties broken towards larger index", "top_budget", _top_ties_reversed),
+    ("forced local diagonals dropped", "select_head", _select_no_force),
+    ("vertical columns left out of the attended set", "attended_mask",
+     _attended_without_verticals),
+]
+
+
+@pytest.mark.parametrize("name,attr,fn", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_mutation_is_caught(monkeypatch, name, attr, fn):
+    monkeypatch.setattr(O, attr, fn)
+    res = _all_checks()
+    failed = [k for k, ok in res.items() if not ok]
+    assert failed, f"no pin caught the planted mistake: {name}"
