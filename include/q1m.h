@@ -1,0 +1,233 @@
+/*
+ * q1m.h — C ABI of the B200 (sm_100a) library for long-context prefill attention of one
+ * grouped-query attention layer: Dual Chunk Attention (DCA) position remapping, YaRN logit
+ * scaling and vertical-slash sparse attention under chunked prefill.
+ *
+ * Sources (page title, section):
+ *   [P2] "Qwen2.5-1M Technical Report" paper review (xllm-io): section 三 (GQA 28/4 and 40/8
+ *        heads, RoPE), section 四 "Dual Chunk Attention" (intra-chunk, inter-chunk and
+ *        successive-chunk patterns; Figure 2: remapped relative positions stay in the trained
+ *        range), "YaRN 注意力缩放" (softmax(q^T k / (t sqrt(D))), sqrt(1/t) = 0.1 ln s + 1),
+ *        "稀疏注意力机制" (MInference vertical-slash; Figure 4: key tokens chosen per prefill
+ *        chunk; continuous relative positions).
+ *   [P5] "Qwen2.5-1M リリース" (agentlenshq): "Sparse Attention" (chunked prefill, 32,768) and
+ *        "Deploy Qwen2.5-1M Models Locally" (--max-num-batched-tokens 131072 = prefill chunk).
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are caller-owned device memory; the library never allocates, frees or
+ *     keeps them. Host pointers are named *_host.
+ *   - Tensors are contiguous. q / out are token-major [seq_len][n_q_heads][head_dim];
+ *     k / v are [seq_len][n_kv_heads][head_dim]; lse is [n_q_heads][seq_len].
+ *   - Arguments are validated synchronously; on failure nothing is launched and a negative
+ *     q1m_status is returned (q1m_last_error() gives a message). Otherwise the work is
+ *     queued on `stream` (a cudaStream_t, NULL = legacy default stream) and the call returns
+ *     Q1M_OK at once. Device-side faults detected by the kernels (a bounded wait that ran
+ *     out, an fp16 range overflow, a NaN score) are latched on the device and returned by
+ *     q1m_status_poll().
+ *   - Calls are thread-safe as long as concurrent calls use distinct workspaces/outputs.
+ *   - head_dim is 64 or 128; n_q_heads is a multiple of n_kv_heads; (dca_chunk - local_window)
+ *     and prefill_chunk are multiples of 128. Only sm_100a devices are supported; there is no
+ *     CPU fallback.
+ */
+#ifndef Q1M_H_
+#define Q1M_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  Q1M_OK = 0,
+  Q1M_ERR_INVALID = -1,      /* a bad argument (null pointer, bad size or shape)          */
+  Q1M_ERR_UNSUPPORTED = -2,  /* a valid case this build does not handle (head_dim, GPU)   */
+  Q1M_ERR_WORKSPACE = -3,    /* workspace too small                                        */
+  Q1M_ERR_CUDA = -4,         /* a CUDA runtime call failed                                 */
+  Q1M_ERR_TIMEOUT = -5,      /* a device-side bounded wait ran out (latched on the device) */
+  Q1M_ERR_RANGE = -6         /* fp16 overflow in the rotation stage, or a NaN score        */
+} q1m_status;
+
+typedef enum { Q1M_BF16 = 0, Q1M_F32 = 1 } q1m_dtype;
+
+/* Layer parameters. Mirrors the pages' deployment knobs: dca_chunk / local_window (DCA),
+ * yarn_s (YaRN ratio s), prefill_chunk (--max-num-batched-tokens) and the vertical-slash
+ * budgets of the sparse estimator. */
+typedef struct {
+  int32_t in_dtype;        /* q1m_dtype of q, k, v                                         */
+  int32_t out_dtype;       /* q1m_dtype of out                                             */
+  double rope_base;        /* RoPE base, theta_f = base^(-2f/D), rotate-half pairing       */
+  double yarn_s;           /* inference/training length ratio; <= 1 disables the scale     */
+  int64_t dca_chunk;       /* c: trained length; one DCA chunk holds c - local_window tokens */
+  int64_t local_window;    /* w: 0 <= w < c                                                */
+  int32_t vs_vertical;     /* vertical budget per head (columns); 0 and 0 => dense         */
+  int32_t vs_slash;        /* slash budget per head (diagonals)                            */
+  int32_t vs_last_q;       /* estimator rows: the last vs_last_q rows of a chunk (1..64)   */
+  int32_t vs_force_local;  /* diagonals 0 .. vs_force_local-1 always kept (>= 1 if sparse) */
+  int64_t prefill_chunk;   /* query rows per chunked-prefill step (multiple of 128)        */
+} q1m_params;
+
+/* ---------------------------------------------------------------------------------------
+ * Whole layer
+ * ------------------------------------------------------------------------------------- */
+
+/* Bytes of device workspace q1m_dca_sparse_prefill needs for this shape (0 on bad input). */
+size_t q1m_workspace_bytes(int64_t seq_len, int n_q_heads, int n_kv_heads, int head_dim,
+                           const q1m_params* p);
+
+/* The layer: for every prefill chunk [s0, e) (s0 = p * prefill_chunk, e = min(N, s0 + P)),
+ * rotate the chunk's keys and queries (DCA views), estimate vertical/slash scores from the
+ * chunk's last vs_last_q rows over keys [0, e), select the per-head budgets, build the
+ * 128 x 128 block mask, run block-sparse DCA attention for rows [s0, e) and merge the three
+ * DCA patterns' partial results ([P2] 四; [P5] Sparse Attention).
+ * q: [N][Hq][D], k, v: [N][Hkv][D] in p->in_dtype; out: [N][Hq][D] in p->out_dtype;
+ * lse (nullable): [Hq][N] fp32, natural-log log-sum-exp of each row's scaled logits.
+ * workspace: device memory of at least q1m_workspace_bytes(...) bytes, 256-byte aligned. */
+q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, void* out,
+                                  float* lse, int64_t seq_len, int n_q_heads, int n_kv_heads,
+                                  int head_dim, const q1m_params* p, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace q1m_dca_sparse_prefill_host needs (staging for q, k, v, out
+ * and lse plus q1m_workspace_bytes). */
+size_t q1m_host_workspace_bytes(int64_t seq_len, int n_q_heads, int n_kv_heads, int head_dim,
+                                const q1m_params* p);
+
+/* The same layer from host buffers: copies q/k/v host->device (cudaMemcpyAsync, one per
+ * tensor), runs q1m_dca_sparse_prefill, copies out (and lse if non-null) back, then
+ * synchronizes `stream`. Host buffers should be pinned for full copy bandwidth. Returns the
+ * device-side status of the run. */
+q1m_status q1m_dca_sparse_prefill_host(const void* q_host, const void* k_host,
+                                       const void* v_host, void* out_host, float* lse_host,
+                                       int64_t seq_len, int n_q_heads, int n_kv_heads,
+                                       int head_dim, const q1m_params* p, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Stages (the same kernels the layer runs; exported for tests and measurement)
+ * ------------------------------------------------------------------------------------- */
+
+/* Cosine/sine table for RoPE positions 0 .. n_pos-1 ([P2] 三 RoPE): table[pos][f] =
+ * (cos, sin)(pos * base^(-2f/D)) as float2, f < D/2, angles formed in fp64.
+ * table: device, n_pos * D/2 float2. */
+q1m_status q1m_rope_table(float* table, int64_t n_pos, int head_dim, double rope_base,
+                          void* stream);
+
+/* DCA key rotation ([P2] 四 DCA: keys sit at position j mod (c - w)) for tokens [s0, e):
+ * k_rot[g][j][:] = fp16(R(j mod L) k[j][g][:]), v16[g][j][:] = fp16(v[j][g][:]).
+ * k_rot, v16: device [Hkv][ld_tokens][D] fp16 (ld_tokens >= e, a multiple of 128).
+ * table: q1m_rope_table output for n_pos >= dca_chunk. Values beyond fp16 range latch
+ * Q1M_ERR_RANGE. */
+q1m_status q1m_rope_dca_keys(const void* k, const void* v, int64_t s0, int64_t e,
+                             int n_kv_heads, int head_dim, const q1m_params* p,
+                             const float* table, uint16_t* k_rot, uint16_t* v16,
+                             int64_t ld_tokens, void* stream);
+
+/* DCA query views for rows [s0, e) ([P2] 四 DCA and YaRN): for pattern x in
+ * {0 intra, 1 successive, 2 inter}, qv[x][h][i - s0][:] = fp16(R(pos_x(i)) q[i][h][:] *
+ * (1/t) / sqrt(D) * log2(e)) with pos_0 = i mod L, pos_1 = min(i mod L + L, c - 1),
+ * pos_2 = c - 1, L = c - w. qv: device [3][Hq][ld_rows][D] fp16 (ld_rows >= e - s0,
+ * multiple of 128; rows e - s0 .. ld_rows-1 are zeroed). */
+q1m_status q1m_rope_dca_queries(const void* q, int64_t s0, int64_t e, int n_q_heads,
+                                int head_dim, const q1m_params* p, const float* table,
+                                uint16_t* qv, int64_t ld_rows, void* stream);
+
+/* Bytes of scratch q1m_vs_estimate needs for a chunk ending at e. */
+size_t q1m_vs_estimate_scratch_bytes(int64_t e, int n_q_heads, int n_kv_heads, int head_dim);
+
+/* Vertical-slash estimator ([P2] 四 稀疏注意力机制; MInference vertical-slash): for the rows
+ * R = [max(s0, e - vs_last_q), e) and each Q head h, p_ij = softmax over j <= i of the DCA
+ * logits; vert[h][j] = sum_{i in R} p_ij and slash[h][o] = sum_{i in R} p_{i,i-o} for
+ * j, o in [0, e). q: raw queries [N][Hq][D] (in_dtype); k_rot: q1m_rope_dca_keys output
+ * covering [0, e). vert, slash: device fp32 [Hq][ld] (ld >= e). scratch: device memory of
+ * q1m_vs_estimate_scratch_bytes(...) bytes. */
+q1m_status q1m_vs_estimate(const void* q, const uint16_t* k_rot, int64_t ld_tokens, int64_t s0,
+                           int64_t e, int n_q_heads, int n_kv_heads, int head_dim,
+                           const q1m_params* p, const float* table, float* vert, float* slash,
+                           int64_t ld, void* scratch, size_t scratch_bytes, void* stream);
+
+/* Bytes of scratch q1m_vs_select needs for candidates [0, e). */
+size_t q1m_vs_select_scratch_bytes(int64_t e, int n_q_heads);
+
+/* Budget selection: per head, the vs_vertical columns with the largest vert score and the
+ * vs_slash offsets with the largest slash score, offsets < vs_force_local always kept;
+ * larger score first, equal scores by smaller index; a budget >= e keeps all. Results are
+ * written in ascending order: V [Hq][min(vs_vertical, e)] and S [Hq][min(vs_slash, e)]
+ * int32 (device). Scores must be >= 0 (NaN latches Q1M_ERR_RANGE). */
+q1m_status q1m_vs_select(const float* vert, const float* slash, int64_t ld, int64_t e,
+                         int n_q_heads, const q1m_params* p, int32_t* V, int32_t* S,
+                         void* scratch, size_t scratch_bytes, void* stream);
+
+/* Block mask and residual verticals for query blocks b of rows [s0, e) (128 x 128 blocks):
+ * key block kb of query block b (rows r0 = 128b .. r1 = min(128b+127, e-1)) is computed when
+ * some o in S has o <= r1 and floor(max(0, r0-o)/128) <= kb <= floor((r1-o)/128); residual
+ * verticals are the j in V with j <= r1 whose block is not computed (ascending).
+ * Outputs (device), nqb = ceil((e - s0)/128), nkw = ceil(ceil(e/128)/32):
+ *   mask  [Hq][nqb][nkw] uint32, bit kb%32 of word kb/32;
+ *   resid [Hq][nqb][nv] int32 (nv = min(vs_vertical, e)), entries past the count undefined;
+ *   cnt   [Hq][nqb][8] int32: computed blocks per DCA pattern (0 intra, 1 successive,
+ *         2 inter), then residual columns per pattern (same order), then total residuals,
+ *         then 0. The ascending residual list holds inter, then successive, then intra. */
+q1m_status q1m_vs_build_masks(const int32_t* V, const int32_t* S, int64_t s0, int64_t e,
+                              int n_q_heads, const q1m_params* p, uint32_t* mask,
+                              int32_t* resid, int32_t* cnt, void* stream);
+
+/* Bytes of scratch q1m_block_sparse_attn needs for rows [s0, e). */
+size_t q1m_attn_scratch_bytes(int64_t s0, int64_t e, int n_q_heads, int head_dim);
+
+/* Block-sparse DCA attention on the tensor cores for rows [s0, e), one partial result per
+ * DCA pattern x (0 intra, 1 successive, 2 inter; query view x): over the keys of that pattern in
+ * A(i) (computed blocks and residual verticals; every causal key when mask == NULL),
+ *   o_part[x][h][i - s0][:] = softmax-weighted sum of v (fp32), lse_part[x][h][i - s0] =
+ *   log2-sum-exp2 of the log2-scaled logits (-inf when the segment is empty for the row).
+ * qv, k_rot, v16: stage outputs above; mask/resid/cnt: q1m_vs_build_masks output or NULL.
+ * o_part: device fp32 [3][Hq][ld_rows][D]; lse_part: device fp32 [3][Hq][ld_rows]. */
+q1m_status q1m_block_sparse_attn(const uint16_t* qv, int64_t ld_rows, const uint16_t* k_rot,
+                                 const uint16_t* v16, int64_t ld_tokens, const uint32_t* mask,
+                                 const int32_t* resid, const int32_t* cnt, int64_t s0,
+                                 int64_t e, int n_q_heads, int n_kv_heads, int head_dim,
+                                 const q1m_params* p, float* o_part, float* lse_part,
+                                 void* scratch, size_t scratch_bytes, void* stream);
+
+/* Log-sum-exp merge of the DCA patterns' partial results for rows [s0, e)
+ * (lse = log2 sum_x 2^lse_x, out = sum_x 2^(lse_x - lse) o_x):
+ * out[i][h][:] in out_dtype ([N][Hq][D] layout) and lse[h][i] (natural log, nullable).
+ * n_parts partials laid out as q1m_block_sparse_attn writes them. With p non-NULL and
+ * n_parts == 3, a row reads only the patterns it has keys in (inter from the third DCA
+ * chunk on, successive from the second), which is what q1m_block_sparse_attn writes;
+ * with p NULL every part is read and an empty part must hold lse = -inf. */
+q1m_status q1m_lse_merge(const float* o_part, const float* lse_part, int n_parts,
+                         int64_t ld_rows, int64_t s0, int64_t e, int64_t seq_len,
+                         int n_q_heads, int head_dim, int out_dtype, const q1m_params* p,
+                         void* out, float* lse, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Status
+ * ------------------------------------------------------------------------------------- */
+
+/* Synchronizes `stream`, then returns and clears the device-side status latched by the
+ * kernels on the current device (Q1M_OK, Q1M_ERR_TIMEOUT or Q1M_ERR_RANGE), or
+ * Q1M_ERR_CUDA if the stream reported an error. */
+q1m_status q1m_status_poll(void* stream);
+
+/* The message of the last failing call on this thread ("" if none). */
+const char* q1m_last_error(void);
+
+/* Library version string. */
+const char* q1m_version(void);
+
+/* Sets the budget, in SM clock cycles, of the kernels' bounded waits on the current device
+ * (default 2e9, about one second); 0 restores the default. */
+q1m_status q1m_set_wait_budget(uint64_t cycles);
+
+/* Self-test of the bounded waits: launches one warp that waits on a barrier nothing ever
+ * arrives on, with a budget of `cycles`, and returns what q1m_status_poll then reports
+ * (Q1M_ERR_TIMEOUT when the wait gave up as designed). The default budget is restored. */
+q1m_status q1m_selftest_wait_timeout(uint64_t cycles, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q1M_H_ */

@@ -1,0 +1,520 @@
+// attn_tc.cuh — block-sparse DCA flash attention on the 5th-generation tensor cores.
+//
+// "Qwen2.5-1M Technical Report" paper review (xllm-io), section 四: DCA's three patterns
+// (intra / successive / inter chunk), MInference vertical-slash sparse attention with key
+// tokens chosen per prefill chunk, and the sparse attention kernel (Figure 7). That
+// kernel was written for A100; this one is designed for sm_100a:
+//
+//  * A work item is (Q head h, a pair of adjacent 128-row query blocks, DCA pattern x).
+//    Pattern x (0 intra, 1 successive, 2 inter) selects the key blocks of that pattern; all
+//    of them use the same rotated query view x, so each item loads one Q view per query
+//    block, and the item writes a partial result (o, log2-sum-exp2) that a separate kernel
+//    merges.
+//  * The two query blocks of an item ("slots") share one stream of K/V tiles: the union of
+//    their key-block lists, each tile flagged with the slots that use it. Slot 1 is the
+//    block right after slot 0, so in dense mode the lists coincide and in sparse mode
+//    (Toeplitz block masks) they mostly do.
+//  * Warp roles: warps 0-3 softmax of slot 0, warps 4-7 softmax of slot 1, warp 8 loads
+//    (TMA for key blocks, cp.async gathers for residual vertical columns), warp 9 issues
+//    tcgen05.mma and owns tensor memory.
+//  * Tensor memory per slot: S (128 fp32 columns), O (D fp32 columns); the softmax writes
+//    P as packed fp16 over the first 64 columns of S and the PV product reads it from
+//    tensor memory (A operand), with V as an MN-major shared-memory operand.
+//  * The MMA warp issues, per tile: [PV of the slot's previous tile] then QK^T of this
+//    tile, alternating slots, so one slot's softmax overlaps the other slot's MMAs.
+//  * Online softmax in base 2 with a lazy rescale: O (in TMEM) and l are rescaled only
+//    when a row's running maximum grows by more than 2^8.
+#pragma once
+
+#include "q1m_device.cuh"
+
+namespace q1m {
+
+constexpr int K3_NK = 2;        // K stages
+constexpr int K3_NV = 2;        // V stages
+constexpr int K3_THREADS = 320;
+constexpr float K3_RESCALE_THRESHOLD = 8.0f;
+
+struct K3Args {
+  int64_t s0, e;
+  int hq, hkv, G;
+  int64_t L;             // DCA chunk length in tokens (multiple of 128)
+  int nqb, npair;
+  int64_t ld_rows, ld_tokens;
+  const uint32_t* mask;  // [hq][nqb][nkw] or null (dense)
+  const int32_t* resid;  // [hq][nqb][nvcap]
+  const int32_t* cnt;    // [hq][nqb][8]
+  int nkw, nvcap;
+  const uint16_t* k_rot;
+  const uint16_t* v16;
+  float* o_part;         // [3][hq][ld_rows][D]
+  float* lse_part;       // [3][hq][ld_rows]
+  const int32_t* units;  // sorted (pair << 2 | pattern)
+  const int32_t* n_units;
+};
+
+struct K3Item {
+  int h, g, x;
+  int qb[2];
+  int64_t B[2];
+  int lo[2], hi[2];      // key-block range of each slot in segment x (lo > hi: empty)
+  int ntiles[2];
+  int nres[2], res_off[2];
+  bool valid[2];
+};
+
+// Key-block range of DCA pattern x for global query block B (Lb blocks per DCA chunk,
+// cb = B / Lb): intra (0) = chunk cb up to the diagonal block B, successive (1) = chunk
+// cb - 1, inter (2) = chunks <= cb - 2. Empty ranges have lo > hi.
+__device__ __forceinline__ void seg_range(int64_t B, int x, int64_t Lb, int* lo, int* hi) {
+  const int64_t cb = B / Lb;
+  if (x == 0) { *lo = (int)(cb * Lb); *hi = (int)B; }
+  else if (x == 1) { if (cb >= 1) { *lo = (int)((cb - 1) * Lb); *hi = (int)(cb * Lb - 1); } else { *lo = 1; *hi = 0; } }
+  else { if (cb >= 2) { *lo = 0; *hi = (int)((cb - 1) * Lb - 1); } else { *lo = 1; *hi = 0; } }
+}
+
+__device__ __forceinline__ K3Item k3_item(const K3Args& a, int it) {
+  K3Item r;
+  const int u = a.units[it / a.hq];
+  r.h = it % a.hq;
+  r.g = r.h / a.G;
+  r.x = u & 3;
+  const int m = u >> 2;
+  const int64_t Lb = a.L / 128;
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    r.qb[s] = 2 * m + s;
+    r.valid[s] = r.qb[s] < a.nqb;
+    r.B[s] = a.s0 / 128 + r.qb[s];
+    r.lo[s] = 1; r.hi[s] = 0; r.ntiles[s] = 0; r.nres[s] = 0; r.res_off[s] = 0;
+    if (!r.valid[s]) continue;
+    seg_range(r.B[s], r.x, Lb, &r.lo[s], &r.hi[s]);
+    if (a.mask == nullptr) {
+      r.ntiles[s] = r.hi[s] >= r.lo[s] ? r.hi[s] - r.lo[s] + 1 : 0;
+    } else {
+      const int32_t* c = a.cnt + ((int64_t)r.h * a.nqb + r.qb[s]) * 8;
+      r.nres[s] = c[3 + r.x];
+      // the ascending residual list holds inter columns, then successive, then intra
+      r.res_off[s] = (r.x < 2 ? c[5] : 0) + (r.x < 1 ? c[4] : 0);
+      r.ntiles[s] = c[r.x] + (r.nres[s] + 127) / 128;
+    }
+  }
+  return r;
+}
+
+__device__ __forceinline__ uint32_t range_bits(int w, int lo, int hi) {
+  if (hi < lo) return 0u;
+  const int b0 = 32 * w, b1 = b0 + 31;
+  if (hi < b0 || lo > b1) return 0u;
+  const int l = lo > b0 ? lo - b0 : 0;
+  const int h = hi < b1 ? hi - b0 : 31;
+  const uint32_t upto = h == 31 ? 0xFFFFFFFFu : ((1u << (h + 1)) - 1u);
+  return upto & ~((1u << l) - 1u);
+}
+
+template <int D>
+struct K3Smem {
+  static constexpr int TILE = 128 * D * 2;  // bytes of one 128-row fp16 tile
+  alignas(1024) uint8_t q[2][TILE];
+  alignas(1024) uint8_t k[K3_NK][TILE];
+  alignas(1024) uint8_t v[K3_NV][TILE];
+  int desc[K3_NK][4];       // flags, diag mask, ncols (gathers; 128 for blocks), unused
+  int meta[2];              // per-slot mailbox written by the MMA warp before its arrive
+  uint64_t k_full[K3_NK], k_empty[K3_NK], v_full[K3_NV], v_empty[K3_NV];
+  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_done[2], pv_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+};
+
+// --------------------------------------------------------------------------------------
+// Loader warp
+// --------------------------------------------------------------------------------------
+template <int D>
+__device__ void k3_gather(K3Smem<D>& sm, const K3Args& a, int g, const int32_t* cols, int n,
+                          int kst, int vst) {
+  // 128 rows x D fp16 of k_rot and v16 gathered by column index into the swizzled layout
+  const uint32_t lane = lane_id();
+  constexpr int CHUNKS = D / 8;  // 16-byte chunks per row
+  for (int r = (int)lane; r < 128; r += 32) {
+    const int j = cols[r < n ? r : 0];
+    const uint16_t* ks = a.k_rot + ((int64_t)g * a.ld_tokens + j) * D;
+    const uint16_t* vs = a.v16 + ((int64_t)g * a.ld_tokens + j) * D;
+#pragma unroll
+    for (int c = 0; c < CHUNKS; ++c) {
+      const uint32_t off = (uint32_t)(c >> 3) * 16384u + sw128_offset((uint32_t)r, (uint32_t)(c & 7));
+      cp_async16(sm.k[kst] + off, ks + c * 8);
+      cp_async16(sm.v[vst] + off, vs + c * 8);
+    }
+  }
+  cp_async_wait_all();
+  fence_async_smem();
+  __syncwarp();
+}
+
+template <int D>
+__device__ void k3_producer(K3Smem<D>& sm, const K3Args& a, const CUtensorMap* mq,
+                            const CUtensorMap* mk, const CUtensorMap* mv, int nitems) {
+  constexpr uint32_t TILE = K3Smem<D>::TILE;
+  const bool leader = lane_id() == 0;
+  uint32_t kt = 0;             // tiles produced by this CTA
+  uint32_t qn[2] = {0, 0};     // Q loads per slot
+  bool ok = true;
+  for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+    const K3Item I = k3_item(a, it);
+    // Q views of both slots
+    for (int s = 0; s < 2 && ok; ++s) {
+      if (I.ntiles[s] == 0) continue;
+      ok = mbar_wait_warp(&sm.q_empty[s], (qn[s] & 1) ^ 1);
+      if (!ok) break;
+      if (leader) {
+        mbar_expect_tx(&sm.q_full[s], TILE);
+        const int y = (int)(((int64_t)I.x * a.hq + I.h) * a.ld_rows + (int64_t)I.qb[s] * 128);
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(sm.q[s] + hf * 16384, mq, &sm.q_full[s], 64 * hf, y);
+      }
+      ++qn[s];
+    }
+    // residual vertical columns, per slot, 128 per gathered tile
+    for (int s = 0; s < 2 && ok; ++s) {
+      if (I.nres[s] == 0) continue;
+      const int32_t* cols = a.resid + ((int64_t)I.h * a.nqb + I.qb[s]) * a.nvcap + I.res_off[s];
+      for (int t0 = 0; t0 < I.nres[s] && ok; t0 += 128) {
+        const int kst = kt % K3_NK, vst = kt % K3_NV;
+        ok = mbar_wait_warp(&sm.k_empty[kst], ((kt / K3_NK) & 1) ^ 1) &&
+             mbar_wait_warp(&sm.v_empty[vst], ((kt / K3_NV) & 1) ^ 1);
+        if (!ok) break;
+        const int n = I.nres[s] - t0 < 128 ? I.nres[s] - t0 : 128;
+        if (leader) {
+          sm.desc[kst][0] = 1 << s;
+          sm.desc[kst][1] = 0;
+          sm.desc[kst][2] = n;
+        }
+        k3_gather<D>(sm, a, I.g, cols + t0, n, kst, vst);
+        if (leader) { mbar_arrive(&sm.k_full[kst]); mbar_arrive(&sm.v_full[vst]); }
+        ++kt;
+      }
+    }
+    // key blocks: union of both slots' lists
+    int lo = 1 << 30, hi = -1;
+    for (int s = 0; s < 2; ++s)
+      if (I.ntiles[s] > 0 && I.hi[s] >= I.lo[s]) { lo = min(lo, I.lo[s]); hi = max(hi, I.hi[s]); }
+    for (int w = lo >> 5; w <= (hi >> 5) && hi >= 0 && ok; ++w) {
+      uint32_t m[2];
+      for (int s = 0; s < 2; ++s) {
+        m[s] = (I.ntiles[s] > 0) ? range_bits(w, I.lo[s], I.hi[s]) : 0u;
+        if (m[s] && a.mask) m[s] &= a.mask[((int64_t)I.h * a.nqb + I.qb[s]) * a.nkw + w];
+      }
+      uint32_t u = m[0] | m[1];
+      while (u && ok) {
+        const int b = __ffs(u) - 1;
+        u &= u - 1;
+        const int kb = 32 * w + b;
+        const int flags = (int)((m[0] >> b) & 1u) | (int)(((m[1] >> b) & 1u) << 1);
+        const int diag = (int)(kb == I.B[0]) | ((int)(kb == I.B[1]) << 1);
+        const int kst = kt % K3_NK, vst = kt % K3_NV;
+        ok = mbar_wait_warp(&sm.k_empty[kst], ((kt / K3_NK) & 1) ^ 1);
+        if (!ok) break;
+        const int y = (int)((int64_t)I.g * a.ld_tokens + (int64_t)kb * 128);
+        if (leader) {
+          sm.desc[kst][0] = flags;
+          sm.desc[kst][1] = diag;
+          sm.desc[kst][2] = 128;
+          mbar_expect_tx(&sm.k_full[kst], TILE);
+#pragma unroll
+          for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(sm.k[kst] + hf * 16384, mk, &sm.k_full[kst], 64 * hf, y);
+        }
+        ok = mbar_wait_warp(&sm.v_empty[vst], ((kt / K3_NV) & 1) ^ 1);
+        if (!ok) break;
+        if (leader) {
+          mbar_expect_tx(&sm.v_full[vst], TILE);
+#pragma unroll
+          for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(sm.v[vst] + hf * 16384, mv, &sm.v_full[vst], 64 * hf, y);
+        }
+        ++kt;
+      }
+    }
+  }
+  if (!ok) {
+    // give copies already issued time to land before the CTA exits (TMA completes in
+    // microseconds and depends on nothing else)
+    const long long t0 = clock64();
+    while (clock64() - t0 < 2000000) __nanosleep(1000);
+  }
+}
+
+// --------------------------------------------------------------------------------------
+// MMA warp (one thread issues)
+// --------------------------------------------------------------------------------------
+template <int D>
+__device__ void k3_mma(K3Smem<D>& sm, const K3Args& a, int nitems) {
+  constexpr uint32_t IDESC_QK = idesc_f16(128, 128, 0);
+  constexpr uint32_t IDESC_PV = idesc_f16(128, D, 1);
+  const uint32_t tb = sm.tmem_base;
+  uint32_t kt = 0;
+  uint32_t qn[2] = {0, 0}, sn[2] = {0, 0}, pn[2] = {0, 0};
+  int pend_v[2] = {-1, -1};     // V stage of the slot's pending PV (-1: none)
+  uint32_t pend_kt[2] = {0, 0};
+  bool pend_last[2] = {false, false};
+  bool o_started[2] = {false, false};
+  uint32_t pvd_issued[2] = {0, 0}, pvd_waited[2] = {0, 0};
+  int v_users[K3_NV] = {};
+  bool ok = true;
+
+  auto issue_pv = [&](int s) -> bool {
+    if (!mbar_wait(&sm.p_full[s], pn[s] & 1)) return false;
+    ++pn[s];
+    const int vst = pend_v[s];
+    if (!mbar_wait(&sm.v_full[vst], (pend_kt[s] / K3_NV) & 1)) return false;
+    tc_fence_after();
+    const uint32_t o_t = tb + 256u * s + 128u, p_t = tb + 256u * s;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t vb = smem_u32(sm.v[vst]) + kk * 2048u;
+      mma_ts(o_t, p_t + kk * 8u, sdesc_sw128(vb, 16384u, 1024u), IDESC_PV,
+             (o_started[s] || kk > 0) ? 1u : 0u);
+    }
+    o_started[s] = true;
+    // P lives in S's columns: the next QK^T of this slot may overwrite them only after
+    // this PV has read them
+    mma_commit(&sm.pv_done[s]);
+    ++pvd_issued[s];
+    if (pend_last[s]) { mma_commit(&sm.o_done[s]); o_started[s] = false; }
+    if (--v_users[vst] == 0) mma_commit(&sm.v_empty[vst]);
+    pend_v[s] = -1;
+    return true;
+  };
+
+  for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+    const K3Item I = k3_item(a, it);
+    int rem[2] = {I.ntiles[0], I.ntiles[1]};
+    bool first[2] = {true, true};
+    while ((rem[0] > 0 || rem[1] > 0) && ok) {
+      const int kst = kt % K3_NK, vst = kt % K3_NV;
+      ok = mbar_wait(&sm.k_full[kst], (kt / K3_NK) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const int flags = sm.desc[kst][0], diag = sm.desc[kst][1], ncols = sm.desc[kst][2];
+      int users = 0;
+      for (int s = 0; s < 2 && ok; ++s) {
+        if (pend_v[s] >= 0) { ok = issue_pv(s); if (!ok) break; }
+        if (!(flags & (1 << s))) continue;
+        if (first[s]) {
+          ok = mbar_wait(&sm.q_full[s], qn[s] & 1);
+          if (!ok) break;
+          ++qn[s];
+          first[s] = false;
+          tc_fence_after();
+        }
+        if (pvd_waited[s] < pvd_issued[s]) {
+          ok = mbar_wait(&sm.pv_done[s], pvd_waited[s] & 1);
+          if (!ok) break;
+          ++pvd_waited[s];
+        }
+        --rem[s];
+        const bool last = rem[s] == 0;
+        sm.meta[s] = ((diag >> s) & 1) | (ncols << 8) | ((int)last << 16);
+        mbar_arrive(&sm.s_full[s]);
+        const uint32_t s_t = tb + 256u * s;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
+          mma_ss(s_t, sdesc_sw128(smem_u32(sm.q[s]) + off, 16u, 1024u),
+                 sdesc_sw128(smem_u32(sm.k[kst]) + off, 16u, 1024u), IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&sm.s_full[s]);
+        ++sn[s];
+        if (last) mma_commit(&sm.q_empty[s]);
+        pend_v[s] = vst;
+        pend_kt[s] = kt;
+        pend_last[s] = last;
+        ++users;
+      }
+      if (!ok) break;
+      v_users[vst] = users;
+      mma_commit(&sm.k_empty[kst]);
+      ++kt;
+    }
+  }
+  for (int s = 0; s < 2 && ok; ++s)
+    if (pend_v[s] >= 0) ok = issue_pv(s);
+  mma_commit(&sm.drain);
+  mbar_wait(&sm.drain, 0);
+}
+
+// --------------------------------------------------------------------------------------
+// Softmax warpgroup of one slot: thread t owns row t of the slot's query block.
+// --------------------------------------------------------------------------------------
+template <int D>
+__device__ void k3_softmax(K3Smem<D>& sm, const K3Args& a, int nitems, int s) {
+  const int t = threadIdx.x - 128 * s;          // row within the query block
+  const uint32_t wq = warp_id() & 3u;           // TMEM lane quarter of this warp
+  const uint32_t tb = sm.tmem_base + ((32u * wq) << 16) + 256u * s;
+  uint32_t sn = 0, on = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+    const K3Item I = k3_item(a, it);
+    if (!I.valid[s]) continue;
+    const int64_t row = I.B[s] * 128 + t;       // global row
+    const int64_t rl = row - a.s0;              // row within the chunk
+    const bool live = row < a.e;
+    float* lse_out = a.lse_part + ((int64_t)I.x * a.hq + I.h) * a.ld_rows + rl;
+    if (I.ntiles[s] == 0) {
+      if (live) *lse_out = -INFINITY;
+      continue;
+    }
+    float m = -INFINITY, l = 0.f;
+    bool o_valid = false;
+    for (int tt = 0; tt < I.ntiles[s]; ++tt) {
+      ok = mbar_wait_warp(&sm.s_full[s], sn & 1);
+      if (!ok) break;
+      ++sn;
+      tc_fence_after();
+      const int meta = sm.meta[s];
+      const bool diag = meta & 1;
+      const int ncols = (meta >> 8) & 0xFF;
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tb + 32u * c, reinterpret_cast<uint32_t*>(x) + 32 * c);
+      if (diag || ncols < 128) {
+        const int lim = diag ? t : ncols - 1;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) if (c > lim) x[c] = -INFINITY;
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      const bool need = mx > m + K3_RESCALE_THRESHOLD;
+      if (__any_sync(0xFFFFFFFFu, need)) {
+        const float m_new = need ? mx : m;
+        const float alpha = need ? ex2(m - m_new) : 1.f;
+        l *= alpha;
+        if (o_valid) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tb + 128u + 32u * c, r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+            tmem_st32(tb + 128u + 32u * c, r);
+          }
+        }
+        m = m_new;
+      }
+      const float mu = m == -INFINITY ? 0.f : m;
+      uint32_t pk[64];
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ex2(x[2 * c] - mu), p1 = ex2(x[2 * c + 1] - mu);
+        sum += p0 + p1;
+        pk[c] = pack_f16x2(p0, p1);
+      }
+      l += sum;
+      tmem_st32(tb, pk);
+      tmem_st32(tb + 32u, pk + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.p_full[s]);
+      o_valid = true;
+    }
+    if (!ok) break;
+    ok = mbar_wait_warp(&sm.o_done[s], on & 1);
+    if (!ok) break;
+    ++on;
+    tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float* dst = a.o_part + (((int64_t)I.x * a.hq + I.h) * a.ld_rows + rl) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tb + 128u + 32u * c, r);
+      if (live) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          float4 v4 = make_float4(__uint_as_float(r[j]) * inv, __uint_as_float(r[j + 1]) * inv,
+                                  __uint_as_float(r[j + 2]) * inv, __uint_as_float(r[j + 3]) * inv);
+          *reinterpret_cast<float4*>(dst + 32 * c + j) = v4;
+        }
+      }
+    }
+    if (live) *lse_out = l > 0.f ? m + __log2f(l) : -INFINITY;
+    tc_fence_before();
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(K3_THREADS, 1)
+block_sparse_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                         const __grid_constant__ CUtensorMap mv, const K3Args a) {
+  extern __shared__ uint8_t k3_raw[];
+  K3Smem<D>& sm = *reinterpret_cast<K3Smem<D>*>((reinterpret_cast<uintptr_t>(k3_raw) + 1023) & ~uintptr_t(1023));
+  const int w = warp_id();
+  const int nitems = (*a.n_units) * a.hq;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < K3_NK; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 1); }
+    for (int i = 0; i < K3_NV; ++i) { mbar_init(&sm.v_full[i], 1); mbar_init(&sm.v_empty[i], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.q_full[s], 1); mbar_init(&sm.q_empty[s], 1);
+      mbar_init(&sm.s_full[s], 2); mbar_init(&sm.p_full[s], 128); mbar_init(&sm.o_done[s], 1);
+      mbar_init(&sm.pv_done[s], 1);
+    }
+    mbar_init(&sm.drain, 1);
+    fence_mbar_init();
+  }
+  if (w == 9) { tmem_alloc(&sm.tmem_base, 512); tmem_relinquish(); }
+  if (w == 8 && lane_id() == 0) { tma_prefetch(&mq); tma_prefetch(&mk); tma_prefetch(&mv); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (w < 8) k3_softmax<D>(sm, a, nitems, w >> 2);
+  else if (w == 8) k3_producer<D>(sm, a, &mq, &mk, &mv, nitems);
+  else if (lane_id() == 0) k3_mma<D>(sm, a, nitems);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (w == 9) { __syncwarp(); tmem_dealloc(sm.tmem_base, 512); }
+}
+
+// --------------------------------------------------------------------------------------
+// Work units: (pair m, pattern x) sorted by dense tile count, largest first, so the
+// static round-robin over (unit, head) items starts with the longest items.
+// --------------------------------------------------------------------------------------
+__global__ void k3_units_kernel(int64_t s0, int nqb, int64_t L, int32_t* units, int32_t* n_units) {
+  const int npair = (nqb + 1) / 2;
+  const int U = 3 * npair;
+  const int64_t Lb = L / 128;
+  extern __shared__ int32_t ucost[];
+  for (int u = threadIdx.x; u < U; u += blockDim.x) {
+    const int m = u / 3, x = u % 3;
+    int c = 0;
+    for (int s = 0; s < 2; ++s) {
+      const int qb = 2 * m + s;
+      if (qb >= nqb) continue;
+      int lo, hi;
+      seg_range(s0 / 128 + qb, x, Lb, &lo, &hi);
+      if (hi >= lo) c = max(c, hi - lo + 1);
+    }
+    ucost[u] = c;
+  }
+  __syncthreads();
+  int nz = 0;
+  for (int u = threadIdx.x; u < U; u += blockDim.x) {
+    const int c = ucost[u];
+    if (c == 0) continue;
+    int rank = 0;
+    for (int v = 0; v < U; ++v) {
+      const int cv = ucost[v];
+      rank += (cv > c) || (cv == c && v < u);
+    }
+    units[rank] = ((u / 3) << 2) | (u % 3);
+    ++nz;
+  }
+  __shared__ int total;
+  if (threadIdx.x == 0) total = 0;
+  __syncthreads();
+  atomicAdd(&total, nz);
+  __syncthreads();
+  if (threadIdx.x == 0) *n_units = total;
+}
+
+}  // namespace q1m

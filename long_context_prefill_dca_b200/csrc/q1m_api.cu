@@ -1,0 +1,640 @@
+// q1m_api.cu — the C ABI declared in include/q1m.h: argument validation, workspace layout,
+// TMA tensor maps, kernel launches and the chunked-prefill driver. The whole library is
+// this one translation unit (the kernels are headers), so the device status word is shared
+// without relocatable device code.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "q1m_device.cuh"
+#include "rope_dca.cuh"
+#include "vs_select.cuh"
+#include "vs_estimate.cuh"
+#include "attn_tc.cuh"
+#include "lse_merge.cuh"
+
+using namespace q1m;
+
+namespace {
+
+thread_local std::string t_err;
+
+q1m_status fail(q1m_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return s;
+}
+
+#define Q1M_CUDA(call)                                                                 \
+  do {                                                                                 \
+    cudaError_t err_ = (call);                                                         \
+    if (err_ != cudaSuccess)                                                           \
+      return fail(Q1M_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(err_));     \
+  } while (0)
+
+#define Q1M_LAUNCHED()                                                                 \
+  do {                                                                                 \
+    cudaError_t err_ = cudaGetLastError();                                             \
+    if (err_ != cudaSuccess)                                                           \
+      return fail(Q1M_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(err_)); \
+  } while (0)
+
+#define Q1M_TRY(expr)                       \
+  do {                                      \
+    q1m_status st_ = (expr);                \
+    if (st_ != Q1M_OK) return st_;          \
+  } while (0)
+
+inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+inline size_t align_up(size_t x) { return (x + 1023) & ~size_t(1023); }
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D fp16 tensor map with 128-byte swizzle: rows of `inner` elements, `rows` rows.
+q1m_status make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                    uint32_t box_inner, uint32_t box_rows) {
+  auto enc = tmap_encode();
+  if (!enc) return fail(Q1M_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return fail(Q1M_ERR_INVALID, "tensor base not 16-byte aligned");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(Q1M_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return Q1M_OK;
+}
+
+struct Dev {
+  int sms = 0;
+  bool sm100 = false;
+};
+
+q1m_status device_info(Dev* d) {
+  int dev = 0;
+  Q1M_CUDA(cudaGetDevice(&dev));
+  int major = 0, minor = 0;
+  Q1M_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  Q1M_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  Q1M_CUDA(cudaDeviceGetAttribute(&d->sms, cudaDevAttrMultiProcessorCount, dev));
+  d->sm100 = (major == 10 && minor == 0);
+  if (!d->sm100) return fail(Q1M_ERR_UNSUPPORTED, "device is sm_%d%d; this library runs on sm_100a only", major, minor);
+  return Q1M_OK;
+}
+
+bool sparse(const q1m_params* p) { return p->vs_vertical != 0 || p->vs_slash != 0; }
+
+q1m_status check_shape(int64_t n, int hq, int hkv, int d, const q1m_params* p) {
+  if (!p) return fail(Q1M_ERR_INVALID, "params is NULL");
+  if (n <= 0) return fail(Q1M_ERR_INVALID, "seq_len must be positive");
+  if (hq <= 0 || hkv <= 0 || hq % hkv != 0) return fail(Q1M_ERR_INVALID, "n_q_heads must be a positive multiple of n_kv_heads");
+  if (d != 64 && d != 128) return fail(Q1M_ERR_UNSUPPORTED, "head_dim %d (64 or 128 supported)", d);
+  if (p->in_dtype != Q1M_BF16 && p->in_dtype != Q1M_F32) return fail(Q1M_ERR_INVALID, "bad in_dtype");
+  if (p->out_dtype != Q1M_BF16 && p->out_dtype != Q1M_F32) return fail(Q1M_ERR_INVALID, "bad out_dtype");
+  if (!(p->rope_base > 1.0) || !std::isfinite(p->rope_base)) return fail(Q1M_ERR_INVALID, "rope_base must be > 1");
+  if (!std::isfinite(p->yarn_s)) return fail(Q1M_ERR_INVALID, "yarn_s must be finite");
+  if (p->local_window < 0 || p->dca_chunk <= p->local_window) return fail(Q1M_ERR_INVALID, "need 0 <= local_window < dca_chunk");
+  if ((p->dca_chunk - p->local_window) % 128 != 0) return fail(Q1M_ERR_UNSUPPORTED, "dca_chunk - local_window must be a multiple of 128");
+  if (p->dca_chunk > (int64_t)1 << 30) return fail(Q1M_ERR_UNSUPPORTED, "dca_chunk too large");
+  if (p->prefill_chunk <= 0 || p->prefill_chunk % 128 != 0) return fail(Q1M_ERR_INVALID, "prefill_chunk must be a positive multiple of 128");
+  if (n > ((int64_t)1 << 31) / 8) return fail(Q1M_ERR_UNSUPPORTED, "seq_len too large");
+  if ((int64_t)hkv * round_up(n, 128) >= ((int64_t)1 << 31)) return fail(Q1M_ERR_UNSUPPORTED, "n_kv_heads * seq_len too large");
+  if (sparse(p)) {
+    if (p->vs_vertical < 0 || p->vs_slash < 1) return fail(Q1M_ERR_INVALID, "sparse mode needs vs_slash >= 1 and vs_vertical >= 0");
+    if (p->vs_force_local < 1) return fail(Q1M_ERR_INVALID, "sparse mode needs vs_force_local >= 1 (every row keeps its diagonal)");
+    if (p->vs_last_q < 1 || p->vs_last_q > 64) return fail(Q1M_ERR_INVALID, "vs_last_q must be in [1, 64]");
+    if ((hq / hkv) * 64 > EB_MAX_ROWS) return fail(Q1M_ERR_UNSUPPORTED, "estimator supports at most 7 Q heads per KV head");
+    if ((round_up(n, 128) / 128 + 31) / 32 > MB_MAX_NKW) return fail(Q1M_ERR_UNSUPPORTED, "seq_len too large for the block mask");
+  }
+  return Q1M_OK;
+}
+
+float view_scale(const q1m_params* p, int d) {
+  const double s = p->yarn_s;
+  double inv_t = 1.0;
+  if (s > 1.0) { const double r = 0.1 * std::log(s) + 1.0; inv_t = r * r; }
+  return (float)(inv_t / std::sqrt((double)d) * 1.4426950408889634);  // * log2(e)
+}
+
+// ---- estimator scratch layout --------------------------------------------------------------
+struct EstLayout {
+  int m_pad, n_mt, nsplit, nkt;
+  size_t est_q, part, lse2, slash_part, total;
+};
+
+EstLayout est_layout(int64_t e, int hq, int hkv, int d) {
+  EstLayout L{};
+  const int G = hq / hkv;
+  L.n_mt = (G * 64 + 127) / 128;
+  L.m_pad = L.n_mt * 128;
+  L.nkt = (int)((e + 127) / 128);
+  int ns = (296 + hkv * L.n_mt - 1) / (hkv * L.n_mt);
+  L.nsplit = ns < 1 ? 1 : (ns > L.nkt ? L.nkt : ns);
+  size_t off = 0;
+  L.est_q = off; off = align_up(off + (size_t)4 * hkv * L.m_pad * d * 2);
+  L.part = off; off = align_up(off + (size_t)hkv * L.m_pad * L.nsplit * sizeof(float2));
+  L.lse2 = off; off = align_up(off + (size_t)hkv * L.m_pad * 4);
+  L.slash_part = off; off = align_up(off + (size_t)hq * L.nkt * EB_U * 4);
+  L.total = off;
+  return L;
+}
+
+// ---- whole-layer workspace layout ---------------------------------------------------------
+struct Layout {
+  int64_t ld_tokens, ld_rows, nqb_max, nkw_max;
+  int nv, ns;
+  size_t table, k_rot, v16, qv, o_part, lse_part, units, vert, slash, est, V, Sx, mask, resid,
+      cnt, total;
+};
+
+Layout layout(int64_t n, int hq, int hkv, int d, const q1m_params* p) {
+  Layout L{};
+  L.ld_tokens = round_up(n, 128);
+  const int64_t P = p->prefill_chunk < n ? p->prefill_chunk : n;
+  L.ld_rows = round_up(P, 128);
+  L.nqb_max = L.ld_rows / 128;
+  L.nkw_max = (L.ld_tokens / 128 + 31) / 32;
+  L.nv = (int)(p->vs_vertical < n ? p->vs_vertical : n);
+  L.ns = (int)(p->vs_slash < n ? p->vs_slash : n);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+  L.table = take((size_t)p->dca_chunk * (d / 2) * sizeof(float2));
+  L.k_rot = take((size_t)hkv * L.ld_tokens * d * 2);
+  L.v16 = take((size_t)hkv * L.ld_tokens * d * 2);
+  L.qv = take((size_t)3 * hq * L.ld_rows * d * 2);
+  L.o_part = take((size_t)3 * hq * L.ld_rows * d * 4);
+  L.lse_part = take((size_t)3 * hq * L.ld_rows * 4);
+  L.units = take((size_t)(3 * (L.nqb_max + 1) / 2 + 8) * 4);
+  if (sparse(p)) {
+    L.vert = take((size_t)hq * L.ld_tokens * 4);
+    L.slash = take((size_t)hq * L.ld_tokens * 4);
+    L.est = take(est_layout(n, hq, hkv, d).total);
+    L.V = take((size_t)hq * (L.nv > 0 ? L.nv : 1) * 4);
+    L.Sx = take((size_t)hq * L.ns * 4);
+    L.mask = take((size_t)hq * L.nqb_max * L.nkw_max * 4);
+    L.resid = take((size_t)hq * L.nqb_max * (L.nv > 0 ? L.nv : 1) * 4);
+    L.cnt = take((size_t)hq * L.nqb_max * 8 * 4);
+  }
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* base, size_t off) { return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off); }
+
+int blocks_for(int64_t n, int threads) { return (int)((n + threads - 1) / threads); }
+
+// ---- stage launchers (arguments already validated) ------------------------------------------
+q1m_status run_rope_table(float* table, int64_t n_pos, int d, double base, cudaStream_t st) {
+  const int64_t n = n_pos * (d / 2);
+  rope_table_kernel<<<blocks_for(n, 256), 256, 0, st>>>(reinterpret_cast<float2*>(table), n_pos, d / 2, base);
+  Q1M_LAUNCHED();
+  return Q1M_OK;
+}
+
+q1m_status run_rope_keys(const void* k, const void* v, int64_t s0, int64_t e, int hkv, int d,
+                         const q1m_params* p, const float* table, uint16_t* k_rot, uint16_t* v16,
+                         int64_t ld_tokens, cudaStream_t st) {
+  const int64_t n = (e - s0) * hkv * (d / 2);
+  const int64_t L = p->dca_chunk - p->local_window;
+  const float2* tb = reinterpret_cast<const float2*>(table);
+  if (p->in_dtype == Q1M_BF16)
+    rope_keys_kernel<__nv_bfloat16><<<blocks_for(n, 256), 256, 0, st>>>(
+        (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, s0, e, hkv, d, L, tb, k_rot, v16, ld_tokens);
+  else
+    rope_keys_kernel<float><<<blocks_for(n, 256), 256, 0, st>>>(
+        (const float*)k, (const float*)v, s0, e, hkv, d, L, tb, k_rot, v16, ld_tokens);
+  Q1M_LAUNCHED();
+  return Q1M_OK;
+}
+
+q1m_status run_rope_queries(const void* q, int64_t s0, int64_t e, int hq, int d, const q1m_params* p,
+                            const float* table, uint16_t* qv, int64_t ld_rows, cudaStream_t st) {
+  const int64_t n = ld_rows * hq * (d / 2);
+  const int64_t L = p->dca_chunk - p->local_window;
+  const float sc = view_scale(p, d);
+  const float2* tb = reinterpret_cast<const float2*>(table);
+  if (p->in_dtype == Q1M_BF16)
+    rope_queries_kernel<__nv_bfloat16><<<blocks_for(n, 256), 256, 0, st>>>(
+        (const __nv_bfloat16*)q, s0, e, hq, d, L, p->dca_chunk, sc, tb, qv, ld_rows);
+  else
+    rope_queries_kernel<float><<<blocks_for(n, 256), 256, 0, st>>>(
+        (const float*)q, s0, e, hq, d, L, p->dca_chunk, sc, tb, qv, ld_rows);
+  Q1M_LAUNCHED();
+  return Q1M_OK;
+}
+
+template <int D>
+q1m_status run_estimate_d(const void* q, const uint16_t* k_rot, int64_t ld_tokens, int64_t s0,
+                          int64_t e, int hq, int hkv, const q1m_params* p, const float* table,
+                          float* vert, float* slash, int64_t ld, void* scratch, const Dev& dev,
+                          cudaStream_t st) {
+  const EstLayout EL = est_layout(e, hq, hkv, D);
+  EstArgs a{};
+  a.r_lo = e - p->vs_last_q > s0 ? e - p->vs_last_q : s0;
+  a.e = e;
+  a.hq = hq; a.hkv = hkv; a.G = hq / hkv;
+  a.L = p->dca_chunk - p->local_window;
+  a.ld_tokens = ld_tokens;
+  a.m_pad = EL.m_pad; a.nkt = EL.nkt; a.n_mt = EL.n_mt; a.nsplit = EL.nsplit;
+  a.c_hi = (e - 1) / a.L;
+  a.part = at<float2>(scratch, EL.part);
+  a.lse2 = at<float>(scratch, EL.lse2);
+  a.vert = vert;
+  a.slash_part = at<float>(scratch, EL.slash_part);
+  a.ld = ld;
+  uint16_t* est_q = at<uint16_t>(scratch, EL.est_q);
+  {
+    const int64_t n = (int64_t)4 * hkv * EL.m_pad * (D / 2);
+    const float sc = view_scale(p, D);
+    const float2* tb = reinterpret_cast<const float2*>(table);
+    if (p->in_dtype == Q1M_BF16)
+      est_queries_kernel<__nv_bfloat16><<<blocks_for(n, 256), 256, 0, st>>>(
+          (const __nv_bfloat16*)q, a.r_lo, e, hq, hkv, D, a.L, p->dca_chunk, sc, tb, est_q, EL.m_pad);
+    else
+      est_queries_kernel<float><<<blocks_for(n, 256), 256, 0, st>>>(
+          (const float*)q, a.r_lo, e, hq, hkv, D, a.L, p->dca_chunk, sc, tb, est_q, EL.m_pad);
+    Q1M_LAUNCHED();
+  }
+  CUtensorMap m_est128, m_est64, m_k;
+  const uint64_t est_rows = (uint64_t)4 * hkv * EL.m_pad;
+  Q1M_TRY(make_map(&m_est128, est_q, D, est_rows, 64, 128));
+  Q1M_TRY(make_map(&m_est64, est_q, D, est_rows, 64, 64));
+  Q1M_TRY(make_map(&m_k, k_rot, D, (uint64_t)hkv * ld_tokens, 64, 128));
+  {
+    const size_t smem = sizeof(EASmem<D>) + 1024;
+    Q1M_CUDA(cudaFuncSetAttribute(est_pass_a_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    est_pass_a_kernel<D><<<hkv * EL.n_mt * EL.nsplit, EA_THREADS, smem, st>>>(m_est128, m_k, a);
+    Q1M_LAUNCHED();
+    est_merge_a_kernel<<<blocks_for((int64_t)hkv * EL.m_pad, 256), 256, 0, st>>>(a);
+    Q1M_LAUNCHED();
+  }
+  {
+    const size_t smem = sizeof(EBSmem<D>) + 1024;
+    Q1M_CUDA(cudaFuncSetAttribute(est_pass_b_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    const int64_t W = (int64_t)hkv * EL.nkt;
+    const int grid = (int)(W < dev.sms ? W : dev.sms);
+    est_pass_b_kernel<D><<<grid, EB_THREADS, smem, st>>>(m_est64, m_k, a);
+    Q1M_LAUNCHED();
+    est_slash_reduce_kernel<<<blocks_for((int64_t)hq * e, 256), 256, 0, st>>>(a, slash);
+    Q1M_LAUNCHED();
+  }
+  return Q1M_OK;
+}
+
+q1m_status run_select(const float* vert, const float* slash, int64_t ld, int64_t e, int hq,
+                      const q1m_params* p, int32_t* V, int32_t* Sx, cudaStream_t st) {
+  vs_select_kernel<<<dim3(hq, 2), SEL_THREADS, 0, st>>>(vert, slash, ld, e, p->vs_vertical,
+                                                       p->vs_slash, p->vs_force_local, V, Sx);
+  Q1M_LAUNCHED();
+  return Q1M_OK;
+}
+
+q1m_status run_masks(const int32_t* V, const int32_t* Sx, int64_t s0, int64_t e, int hq,
+                     const q1m_params* p, uint32_t* mask, int32_t* resid, int32_t* cnt,
+                     cudaStream_t st) {
+  const int nqb = (int)((e - s0 + 127) / 128);
+  const int nv = (int)(p->vs_vertical < e ? p->vs_vertical : e);
+  const int ns = (int)(p->vs_slash < e ? p->vs_slash : e);
+  vs_mask_kernel<<<dim3(hq, (nqb + MB_QB - 1) / MB_QB), MB_THREADS, 0, st>>>(
+      V, Sx, s0, e, nv, ns, p->dca_chunk - p->local_window, mask, resid, cnt);
+  Q1M_LAUNCHED();
+  return Q1M_OK;
+}
+
+template <int D>
+q1m_status run_attn_d(const uint16_t* qv, int64_t ld_rows, const uint16_t* k_rot, const uint16_t* v16,
+                      int64_t ld_tokens, const uint32_t* mask, const int32_t* resid, const int32_t* cnt,
+                      int64_t s0, int64_t e, int hq, int hkv, const q1m_params* p, float* o_part,
+                      float* lse_part, int32_t* units, const Dev& dev, cudaStream_t st) {
+  K3Args a{};
+  a.s0 = s0; a.e = e; a.hq = hq; a.hkv = hkv; a.G = hq / hkv;
+  a.L = p->dca_chunk - p->local_window;
+  a.nqb = (int)((e - s0 + 127) / 128);
+  a.npair = (a.nqb + 1) / 2;
+  a.ld_rows = ld_rows; a.ld_tokens = ld_tokens;
+  a.mask = mask; a.resid = resid; a.cnt = cnt;
+  a.nkw = (int)(((e + 127) / 128 + 31) / 32);
+  a.nvcap = (int)(p->vs_vertical < e ? p->vs_vertical : e);
+  a.k_rot = k_rot; a.v16 = v16;
+  a.o_part = o_part; a.lse_part = lse_part;
+  a.units = units + 8;
+  a.n_units = units;
+  const int U = 3 * a.npair;
+  k3_units_kernel<<<1, 1024, (size_t)U * 4, st>>>(s0, a.nqb, a.L, units + 8, units);
+  Q1M_LAUNCHED();
+  CUtensorMap mq, mk, mv;
+  Q1M_TRY(make_map(&mq, qv, D, (uint64_t)3 * hq * ld_rows, 64, 128));
+  Q1M_TRY(make_map(&mk, k_rot, D, (uint64_t)hkv * ld_tokens, 64, 128));
+  Q1M_TRY(make_map(&mv, v16, D, (uint64_t)hkv * ld_tokens, 64, 128));
+  const size_t smem = sizeof(K3Smem<D>) + 1024;
+  Q1M_CUDA(cudaFuncSetAttribute(block_sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int64_t items_max = (int64_t)U * hq;
+  const int grid = (int)(items_max < dev.sms ? items_max : dev.sms);
+  block_sparse_attn_kernel<D><<<grid, K3_THREADS, smem, st>>>(mq, mk, mv, a);
+  Q1M_LAUNCHED();
+  return Q1M_OK;
+}
+
+q1m_status run_merge(const float* o_part, const float* lse_part, int n_parts, int64_t ld_rows,
+                     int64_t s0, int64_t e, int64_t n, int hq, int d, int out_dtype, int64_t L,
+                     void* out, float* lse, cudaStream_t st) {
+  const int64_t warps = (e - s0) * hq;
+  const int grid = blocks_for(warps * 32, 256);
+  if (out_dtype == Q1M_BF16) {
+    if (d == 128) lse_merge_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(o_part, lse_part, n_parts, ld_rows, s0, e, hq, L, (__nv_bfloat16*)out, lse, n);
+    else lse_merge_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(o_part, lse_part, n_parts, ld_rows, s0, e, hq, L, (__nv_bfloat16*)out, lse, n);
+  } else {
+    if (d == 128) lse_merge_kernel<float, 128><<<grid, 256, 0, st>>>(o_part, lse_part, n_parts, ld_rows, s0, e, hq, L, (float*)out, lse, n);
+    else lse_merge_kernel<float, 64><<<grid, 256, 0, st>>>(o_part, lse_part, n_parts, ld_rows, s0, e, hq, L, (float*)out, lse, n);
+  }
+  Q1M_LAUNCHED();
+  return Q1M_OK;
+}
+
+}  // namespace
+
+// =============================================================================================
+// C ABI
+// =============================================================================================
+extern "C" {
+
+const char* q1m_version(void) { return "q1m 0.1 (sm_100a)"; }
+
+const char* q1m_last_error(void) { return t_err.c_str(); }
+
+size_t q1m_workspace_bytes(int64_t n, int hq, int hkv, int d, const q1m_params* p) {
+  if (check_shape(n, hq, hkv, d, p) != Q1M_OK) return 0;
+  return layout(n, hq, hkv, d, p).total;
+}
+
+size_t q1m_host_workspace_bytes(int64_t n, int hq, int hkv, int d, const q1m_params* p) {
+  if (check_shape(n, hq, hkv, d, p) != Q1M_OK) return 0;
+  const size_t ein = p->in_dtype == Q1M_BF16 ? 2 : 4, eout = p->out_dtype == Q1M_BF16 ? 2 : 4;
+  return align_up((size_t)n * hq * d * ein) + 2 * align_up((size_t)n * hkv * d * ein) +
+         align_up((size_t)n * hq * d * eout) + align_up((size_t)n * hq * 4) +
+         layout(n, hq, hkv, d, p).total;
+}
+
+q1m_status q1m_rope_table(float* table, int64_t n_pos, int d, double base, void* stream) {
+  if (!table || n_pos <= 0) return fail(Q1M_ERR_INVALID, "bad table arguments");
+  if (d != 64 && d != 128) return fail(Q1M_ERR_UNSUPPORTED, "head_dim %d", d);
+  if (!(base > 1.0)) return fail(Q1M_ERR_INVALID, "rope_base must be > 1");
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  return run_rope_table(table, n_pos, d, base, S(stream));
+}
+
+q1m_status q1m_rope_dca_keys(const void* k, const void* v, int64_t s0, int64_t e, int hkv, int d,
+                             const q1m_params* p, const float* table, uint16_t* k_rot, uint16_t* v16,
+                             int64_t ld_tokens, void* stream) {
+  Q1M_TRY(check_shape(e > 0 ? e : 1, hkv, hkv, d, p));
+  if (!k || !v || !table || !k_rot || !v16) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (s0 < 0 || e <= s0 || ld_tokens < e || ld_tokens % 128) return fail(Q1M_ERR_INVALID, "bad token range");
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  return run_rope_keys(k, v, s0, e, hkv, d, p, table, k_rot, v16, ld_tokens, S(stream));
+}
+
+q1m_status q1m_rope_dca_queries(const void* q, int64_t s0, int64_t e, int hq, int d,
+                                const q1m_params* p, const float* table, uint16_t* qv,
+                                int64_t ld_rows, void* stream) {
+  Q1M_TRY(check_shape(e > 0 ? e : 1, hq, hq, d, p));
+  if (!q || !table || !qv) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (s0 < 0 || e <= s0 || ld_rows < e - s0 || ld_rows % 128) return fail(Q1M_ERR_INVALID, "bad row range");
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  return run_rope_queries(q, s0, e, hq, d, p, table, qv, ld_rows, S(stream));
+}
+
+size_t q1m_vs_estimate_scratch_bytes(int64_t e, int hq, int hkv, int d) {
+  if (e <= 0 || hq <= 0 || hkv <= 0 || hq % hkv || (d != 64 && d != 128)) return 0;
+  return est_layout(e, hq, hkv, d).total;
+}
+
+q1m_status q1m_vs_estimate(const void* q, const uint16_t* k_rot, int64_t ld_tokens, int64_t s0,
+                           int64_t e, int hq, int hkv, int d, const q1m_params* p, const float* table,
+                           float* vert, float* slash, int64_t ld, void* scratch, size_t scratch_bytes,
+                           void* stream) {
+  Q1M_TRY(check_shape(e > 0 ? e : 1, hq, hkv, d, p));
+  if (!sparse(p)) return fail(Q1M_ERR_INVALID, "estimator needs a sparse budget");
+  if (!q || !k_rot || !table || !vert || !slash || !scratch) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (s0 < 0 || e <= s0 || ld < e || ld_tokens < e || ld_tokens % 128) return fail(Q1M_ERR_INVALID, "bad range");
+  if (scratch_bytes < q1m_vs_estimate_scratch_bytes(e, hq, hkv, d)) return fail(Q1M_ERR_WORKSPACE, "estimator scratch too small");
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  if (d == 128) return run_estimate_d<128>(q, k_rot, ld_tokens, s0, e, hq, hkv, p, table, vert, slash, ld, scratch, dev, S(stream));
+  return run_estimate_d<64>(q, k_rot, ld_tokens, s0, e, hq, hkv, p, table, vert, slash, ld, scratch, dev, S(stream));
+}
+
+size_t q1m_vs_select_scratch_bytes(int64_t e, int hq) { (void)e; (void)hq; return 0; }
+
+q1m_status q1m_vs_select(const float* vert, const float* slash, int64_t ld, int64_t e, int hq,
+                         const q1m_params* p, int32_t* V, int32_t* Sx, void* scratch,
+                         size_t scratch_bytes, void* stream) {
+  (void)scratch; (void)scratch_bytes;
+  if (!p || !vert || !slash || !Sx || (p->vs_vertical > 0 && !V)) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (e <= 0 || ld < e || hq <= 0) return fail(Q1M_ERR_INVALID, "bad sizes");
+  if (p->vs_vertical < 0 || p->vs_slash < 1 || p->vs_force_local < 0) return fail(Q1M_ERR_INVALID, "bad budgets");
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  return run_select(vert, slash, ld, e, hq, p, V, Sx, S(stream));
+}
+
+q1m_status q1m_vs_build_masks(const int32_t* V, const int32_t* Sx, int64_t s0, int64_t e, int hq,
+                              const q1m_params* p, uint32_t* mask, int32_t* resid, int32_t* cnt,
+                              void* stream) {
+  if (!p || !Sx || !mask || !cnt || (p->vs_vertical > 0 && (!V || !resid))) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (s0 < 0 || e <= s0 || s0 % 128 || hq <= 0) return fail(Q1M_ERR_INVALID, "bad range");
+  if (p->dca_chunk <= p->local_window || (p->dca_chunk - p->local_window) % 128) return fail(Q1M_ERR_UNSUPPORTED, "DCA chunk length must be a multiple of 128");
+  if (((e + 127) / 128 + 31) / 32 > MB_MAX_NKW) return fail(Q1M_ERR_UNSUPPORTED, "too many key blocks");
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  return run_masks(V, Sx, s0, e, hq, p, mask, resid, cnt, S(stream));
+}
+
+size_t q1m_attn_scratch_bytes(int64_t s0, int64_t e, int hq, int d) {
+  (void)hq; (void)d;
+  if (e <= s0) return 0;
+  const int64_t nqb = (e - s0 + 127) / 128;
+  return (size_t)(3 * (nqb + 1) / 2 + 8) * 4;
+}
+
+q1m_status q1m_block_sparse_attn(const uint16_t* qv, int64_t ld_rows, const uint16_t* k_rot,
+                                 const uint16_t* v16, int64_t ld_tokens, const uint32_t* mask,
+                                 const int32_t* resid, const int32_t* cnt, int64_t s0, int64_t e,
+                                 int hq, int hkv, int d, const q1m_params* p, float* o_part,
+                                 float* lse_part, void* scratch, size_t scratch_bytes, void* stream) {
+  Q1M_TRY(check_shape(e > 0 ? e : 1, hq, hkv, d, p));
+  if (!qv || !k_rot || !v16 || !o_part || !lse_part || !scratch) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (mask && (!cnt || (p->vs_vertical > 0 && !resid))) return fail(Q1M_ERR_INVALID, "mask without counts/residuals");
+  if (s0 < 0 || e <= s0 || s0 % 128 || ld_rows < e - s0 || ld_rows % 128 || ld_tokens < e || ld_tokens % 128)
+    return fail(Q1M_ERR_INVALID, "bad range");
+  if (scratch_bytes < q1m_attn_scratch_bytes(s0, e, hq, d)) return fail(Q1M_ERR_WORKSPACE, "attention scratch too small");
+  if (reinterpret_cast<uintptr_t>(scratch) & 3) return fail(Q1M_ERR_INVALID, "scratch misaligned");
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  int32_t* units = static_cast<int32_t*>(scratch);
+  if (d == 128) return run_attn_d<128>(qv, ld_rows, k_rot, v16, ld_tokens, mask, resid, cnt, s0, e, hq, hkv, p, o_part, lse_part, units, dev, S(stream));
+  return run_attn_d<64>(qv, ld_rows, k_rot, v16, ld_tokens, mask, resid, cnt, s0, e, hq, hkv, p, o_part, lse_part, units, dev, S(stream));
+}
+
+q1m_status q1m_lse_merge(const float* o_part, const float* lse_part, int n_parts, int64_t ld_rows,
+                         int64_t s0, int64_t e, int64_t n, int hq, int d, int out_dtype,
+                         const q1m_params* p, void* out, float* lse, void* stream) {
+  if (!o_part || !lse_part || !out) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (n_parts < 1 || n_parts > 3) return fail(Q1M_ERR_INVALID, "n_parts must be 1..3");
+  if (s0 < 0 || e <= s0 || e > n || ld_rows < e - s0 || hq <= 0) return fail(Q1M_ERR_INVALID, "bad range");
+  if (d != 64 && d != 128) return fail(Q1M_ERR_UNSUPPORTED, "head_dim %d", d);
+  if (out_dtype != Q1M_BF16 && out_dtype != Q1M_F32) return fail(Q1M_ERR_INVALID, "bad out_dtype");
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  const int64_t Ld = p ? p->dca_chunk - p->local_window : 0;
+  if (p && Ld <= 0) return fail(Q1M_ERR_INVALID, "bad DCA chunk length");
+  return run_merge(o_part, lse_part, n_parts, ld_rows, s0, e, n, hq, d, out_dtype, Ld, out, lse, S(stream));
+}
+
+q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, void* out,
+                                  float* lse, int64_t n, int hq, int hkv, int d,
+                                  const q1m_params* p, void* ws, size_t ws_bytes, void* stream) {
+  Q1M_TRY(check_shape(n, hq, hkv, d, p));
+  if (!q || !k || !v || !out || !ws) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(Q1M_ERR_INVALID, "workspace must be 256-byte aligned");
+  const Layout L = layout(n, hq, hkv, d, p);
+  if (ws_bytes < L.total) return fail(Q1M_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  cudaStream_t st = S(stream);
+  float* table = at<float>(ws, L.table);
+  uint16_t* k_rot = at<uint16_t>(ws, L.k_rot);
+  uint16_t* v16 = at<uint16_t>(ws, L.v16);
+  uint16_t* qv = at<uint16_t>(ws, L.qv);
+  float* o_part = at<float>(ws, L.o_part);
+  float* lse_part = at<float>(ws, L.lse_part);
+  int32_t* units = at<int32_t>(ws, L.units);
+  const int64_t Ld = p->dca_chunk - p->local_window;
+  Q1M_TRY(run_rope_table(table, p->dca_chunk, d, p->rope_base, st));
+  if (L.ld_tokens > n) {
+    // zero the padded key rows once so tiles past the end read finite values
+    for (int g = 0; g < hkv; ++g) {
+      Q1M_CUDA(cudaMemsetAsync(k_rot + ((int64_t)g * L.ld_tokens + n) * d, 0, (size_t)(L.ld_tokens - n) * d * 2, st));
+      Q1M_CUDA(cudaMemsetAsync(v16 + ((int64_t)g * L.ld_tokens + n) * d, 0, (size_t)(L.ld_tokens - n) * d * 2, st));
+    }
+  }
+  for (int64_t s0 = 0; s0 < n; s0 += p->prefill_chunk) {
+    const int64_t e = s0 + p->prefill_chunk < n ? s0 + p->prefill_chunk : n;
+    Q1M_TRY(run_rope_keys(k, v, s0, e, hkv, d, p, table, k_rot, v16, L.ld_tokens, st));
+    Q1M_TRY(run_rope_queries(q, s0, e, hq, d, p, table, qv, L.ld_rows, st));
+    const uint32_t* mask = nullptr;
+    const int32_t *resid = nullptr, *cnt = nullptr;
+    if (sparse(p)) {
+      float* vert = at<float>(ws, L.vert);
+      float* slash = at<float>(ws, L.slash);
+      int32_t* V = at<int32_t>(ws, L.V);
+      int32_t* Sx = at<int32_t>(ws, L.Sx);
+      if (d == 128) Q1M_TRY(run_estimate_d<128>(q, k_rot, L.ld_tokens, s0, e, hq, hkv, p, table, vert, slash, L.ld_tokens, at<void>(ws, L.est), dev, st));
+      else Q1M_TRY(run_estimate_d<64>(q, k_rot, L.ld_tokens, s0, e, hq, hkv, p, table, vert, slash, L.ld_tokens, at<void>(ws, L.est), dev, st));
+      Q1M_TRY(run_select(vert, slash, L.ld_tokens, e, hq, p, V, Sx, st));
+      Q1M_TRY(run_masks(V, Sx, s0, e, hq, p, at<uint32_t>(ws, L.mask), at<int32_t>(ws, L.resid), at<int32_t>(ws, L.cnt), st));
+      mask = at<uint32_t>(ws, L.mask);
+      resid = at<int32_t>(ws, L.resid);
+      cnt = at<int32_t>(ws, L.cnt);
+    }
+    if (d == 128) Q1M_TRY(run_attn_d<128>(qv, L.ld_rows, k_rot, v16, L.ld_tokens, mask, resid, cnt, s0, e, hq, hkv, p, o_part, lse_part, units, dev, st));
+    else Q1M_TRY(run_attn_d<64>(qv, L.ld_rows, k_rot, v16, L.ld_tokens, mask, resid, cnt, s0, e, hq, hkv, p, o_part, lse_part, units, dev, st));
+    Q1M_TRY(run_merge(o_part, lse_part, 3, L.ld_rows, s0, e, n, hq, d, p->out_dtype, Ld, out, lse, st));
+  }
+  return Q1M_OK;
+}
+
+q1m_status q1m_dca_sparse_prefill_host(const void* q_h, const void* k_h, const void* v_h, void* out_h,
+                                       float* lse_h, int64_t n, int hq, int hkv, int d,
+                                       const q1m_params* p, void* ws, size_t ws_bytes, void* stream) {
+  Q1M_TRY(check_shape(n, hq, hkv, d, p));
+  if (!q_h || !k_h || !v_h || !out_h || !ws) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(Q1M_ERR_INVALID, "workspace must be 256-byte aligned");
+  if (ws_bytes < q1m_host_workspace_bytes(n, hq, hkv, d, p)) return fail(Q1M_ERR_WORKSPACE, "host-path workspace too small");
+  const size_t ein = p->in_dtype == Q1M_BF16 ? 2 : 4, eout = p->out_dtype == Q1M_BF16 ? 2 : 4;
+  const size_t bq = (size_t)n * hq * d * ein, bk = (size_t)n * hkv * d * ein, bo = (size_t)n * hq * d * eout;
+  size_t off = 0;
+  void* dq = at<void>(ws, off); off += align_up(bq);
+  void* dk = at<void>(ws, off); off += align_up(bk);
+  void* dv = at<void>(ws, off); off += align_up(bk);
+  void* dout = at<void>(ws, off); off += align_up(bo);
+  float* dlse = at<float>(ws, off); off += align_up((size_t)n * hq * 4);
+  cudaStream_t st = S(stream);
+  Q1M_CUDA(cudaMemcpyAsync(dq, q_h, bq, cudaMemcpyHostToDevice, st));
+  Q1M_CUDA(cudaMemcpyAsync(dk, k_h, bk, cudaMemcpyHostToDevice, st));
+  Q1M_CUDA(cudaMemcpyAsync(dv, v_h, bk, cudaMemcpyHostToDevice, st));
+  Q1M_TRY(q1m_dca_sparse_prefill(dq, dk, dv, dout, lse_h ? dlse : nullptr, n, hq, hkv, d, p,
+                                 at<void>(ws, off), ws_bytes - off, stream));
+  Q1M_CUDA(cudaMemcpyAsync(out_h, dout, bo, cudaMemcpyDeviceToHost, st));
+  if (lse_h) Q1M_CUDA(cudaMemcpyAsync(lse_h, dlse, (size_t)n * hq * 4, cudaMemcpyDeviceToHost, st));
+  return q1m_status_poll(stream);
+}
+
+q1m_status q1m_status_poll(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(S(stream));
+  if (e != cudaSuccess) return fail(Q1M_ERR_CUDA, "stream error: %s", cudaGetErrorString(e));
+  int st = 0;
+  Q1M_CUDA(cudaMemcpyFromSymbol(&st, g_status, sizeof(int)));
+  if (st != 0) {
+    const int zero = 0;
+    Q1M_CUDA(cudaMemcpyToSymbol(g_status, &zero, sizeof(int)));
+    return fail((q1m_status)st, st == Q1M_ERR_TIMEOUT ? "a device-side wait ran out" : "device-side range/NaN check failed");
+  }
+  return Q1M_OK;
+}
+
+q1m_status q1m_set_wait_budget(uint64_t cycles) {
+  unsigned long long v = cycles ? (unsigned long long)cycles : 2000000000ull;
+  Q1M_CUDA(cudaMemcpyToSymbol(g_wait_cycles, &v, sizeof v));
+  return Q1M_OK;
+}
+
+}  // extern "C"
+
+namespace {
+// one warp waits on a barrier that no thread and no copy ever arrives on
+__global__ void selftest_wait_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) { mbar_init(&bar, 1); fence_mbar_init(); }
+  __syncwarp();
+  mbar_wait(&bar, 0);
+}
+}  // namespace
+
+extern "C" q1m_status q1m_selftest_wait_timeout(uint64_t cycles, void* stream) {
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  Q1M_TRY(q1m_status_poll(stream));
+  Q1M_TRY(q1m_set_wait_budget(cycles ? cycles : 1000000ull));
+  selftest_wait_kernel<<<1, 32, 0, S(stream)>>>();
+  Q1M_LAUNCHED();
+  const q1m_status st = q1m_status_poll(stream);
+  Q1M_TRY(q1m_set_wait_budget(0));
+  return st;
+}

@@ -1,0 +1,157 @@
+// rope_dca.cuh — RoPE table and DCA position remap (rotation of keys and query views).
+//
+// "Qwen2.5-1M Technical Report" paper review (xllm-io), section 三: RoPE; section 四
+// "Dual Chunk Attention": intra-chunk, successive-chunk and inter-chunk patterns keep
+// remapped relative positions inside the trained range; "YaRN 注意力缩放": logits are
+// scaled by (0.1 ln s + 1)^2 / sqrt(D).
+//
+// Positions (one DCA chunk holds L = c - w tokens, c = dca_chunk, w = local_window):
+//   key j                         -> j mod L
+//   query i, intra pattern        -> i mod L
+//   query i, successive pattern   -> min(i mod L + L, c - 1)
+//   query i, inter pattern        -> c - 1
+// RoPE is the rotate-half form on pairs (f, f + D/2), theta_f = base^(-2f/D).
+// Query views carry the whole logit scale (1/t) / sqrt(D) * log2(e), so the attention
+// kernels work in base-2 exponentials directly.
+#pragma once
+
+#include "q1m_device.cuh"
+
+namespace q1m {
+
+enum : int { VIEW_INTRA = 0, VIEW_SUCC = 1, VIEW_INTER = 2 };
+
+template <typename T>
+__device__ __forceinline__ float load_as_f32(const T* p);
+template <>
+__device__ __forceinline__ float load_as_f32<float>(const float* p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float load_as_f32<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+
+__device__ __forceinline__ uint16_t to_f16_checked(float x) {
+  if (!(fabsf(x) <= 65504.f)) latch(Q1M_ERR_RANGE);   // also catches NaN
+  return __half_as_ushort(__float2half_rn(x));
+}
+
+// table[pos][f] = (cos, sin)(pos * base^(-2f/D)), angle in fp64.
+__global__ void rope_table_kernel(float2* table, int64_t n_pos, int half_d, double base) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n_pos * half_d) return;
+  const int64_t pos = idx / half_d;
+  const int f = (int)(idx % half_d);
+  const double theta = pow(base, -2.0 * (double)f / (double)(2 * half_d));
+  double s, c;
+  sincos((double)pos * theta, &s, &c);
+  table[idx] = make_float2((float)c, (float)s);
+}
+
+// Keys [s0, e): k_rot[g][j] = R(j mod L) k[j][g]; v16[g][j] = v[j][g]; fp16.
+template <typename T>
+__global__ void rope_keys_kernel(const T* __restrict__ k, const T* __restrict__ v, int64_t s0,
+                                 int64_t e, int hkv, int d, int64_t L,
+                                 const float2* __restrict__ table, uint16_t* __restrict__ k_rot,
+                                 uint16_t* __restrict__ v16, int64_t ld_tokens) {
+  const int hd = d >> 1;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (e - s0) * hkv * hd;
+  if (idx >= total) return;
+  const int f = (int)(idx % hd);
+  const int g = (int)((idx / hd) % hkv);
+  const int64_t j = s0 + idx / ((int64_t)hd * hkv);
+  const int64_t src = (j * hkv + g) * d;
+  const float x1 = load_as_f32(k + src + f), x2 = load_as_f32(k + src + f + hd);
+  const float2 cs = table[(j % L) * hd + f];
+  const int64_t dst = ((int64_t)g * ld_tokens + j) * d;
+  k_rot[dst + f] = to_f16_checked(x1 * cs.x - x2 * cs.y);
+  k_rot[dst + f + hd] = to_f16_checked(x2 * cs.x + x1 * cs.y);
+  v16[dst + f] = to_f16_checked(load_as_f32(v + src + f));
+  v16[dst + f + hd] = to_f16_checked(load_as_f32(v + src + f + hd));
+}
+
+__device__ __forceinline__ int64_t dca_query_pos(int64_t i, int view, int64_t L, int64_t c) {
+  const int64_t t = i % L;
+  if (view == VIEW_INTRA) return t;
+  if (view == VIEW_SUCC) return t + L < c - 1 ? t + L : c - 1;
+  return c - 1;
+}
+
+// Query views for rows [s0, e): qv[x][h][i - s0] = scale * R(pos_x(i)) q[i][h]; rows
+// e - s0 .. ld_rows-1 are zero.
+template <typename T>
+__global__ void rope_queries_kernel(const T* __restrict__ q, int64_t s0, int64_t e, int hq,
+                                    int d, int64_t L, int64_t c, float scale,
+                                    const float2* __restrict__ table, uint16_t* __restrict__ qv,
+                                    int64_t ld_rows) {
+  const int hd = d >> 1;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = ld_rows * hq * hd;
+  if (idx >= total) return;
+  const int f = (int)(idx % hd);
+  const int h = (int)((idx / hd) % hq);
+  const int64_t r = idx / ((int64_t)hd * hq);
+  const int64_t i = s0 + r;
+  float x1 = 0.f, x2 = 0.f;
+  if (i < e) {
+    const int64_t src = (i * hq + h) * d;
+    x1 = load_as_f32(q + src + f) * scale;
+    x2 = load_as_f32(q + src + f + hd) * scale;
+  }
+#pragma unroll
+  for (int x = 0; x < 3; ++x) {
+    const int64_t dst = (((int64_t)x * hq + h) * ld_rows + r) * d;
+    uint16_t y1 = 0, y2 = 0;
+    if (i < e) {
+      const float2 cs = table[dca_query_pos(i, x, L, c) * hd + f];
+      y1 = to_f16_checked(x1 * cs.x - x2 * cs.y);
+      y2 = to_f16_checked(x2 * cs.x + x1 * cs.y);
+    }
+    qv[dst + f] = y1;
+    qv[dst + f + hd] = y2;
+  }
+}
+
+// Estimator query operand. Rows R = [r_lo, e) (n_r <= 64 rows) of the Q heads of each KV
+// group g are laid out as m = hh * 64 + r (hh < G). For a key block whose DCA chunk is
+// kc, let cls = min(C_hi - kc, 3) with C_hi the chunk of row e - 1; row i then uses the
+// view of pattern chunk(i) - kc = chunk(i) - C_hi + cls (no view, zero row, when that is
+// negative: every key of the block is then in the row's future). Output
+// est_q[cls][g][m][D] fp16, rows m >= G*64 padded with zeros up to m_pad.
+template <typename T>
+__global__ void est_queries_kernel(const T* __restrict__ q, int64_t r_lo, int64_t e, int hq,
+                                   int hkv, int d, int64_t L, int64_t c, float scale,
+                                   const float2* __restrict__ table, uint16_t* __restrict__ est_q,
+                                   int m_pad) {
+  const int hd = d >> 1;
+  const int G = hq / hkv;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)4 * hkv * m_pad * hd;
+  if (idx >= total) return;
+  const int f = (int)(idx % hd);
+  const int m = (int)((idx / hd) % m_pad);
+  const int g = (int)((idx / ((int64_t)hd * m_pad)) % hkv);
+  const int cls = (int)(idx / ((int64_t)hd * m_pad * hkv));
+  const int hh = m / 64, r = m % 64;
+  const int64_t i = r_lo + r;
+  uint16_t y1 = 0, y2 = 0;
+  if (hh < G && i < e) {
+    const int64_t c_hi = (e - 1) / L;
+    const int64_t rel = i / L - c_hi + cls;
+    if (rel >= 0) {
+      const int view = rel == 0 ? VIEW_INTRA : (rel == 1 ? VIEW_SUCC : VIEW_INTER);
+      const int h = g * G + hh;
+      const int64_t src = (i * hq + h) * d;
+      const float x1 = load_as_f32(q + src + f) * scale;
+      const float x2 = load_as_f32(q + src + f + hd) * scale;
+      const float2 cs = table[dca_query_pos(i, view, L, c) * hd + f];
+      y1 = to_f16_checked(x1 * cs.x - x2 * cs.y);
+      y2 = to_f16_checked(x2 * cs.x + x1 * cs.y);
+    }
+  }
+  const int64_t dst = (((int64_t)cls * hkv + g) * m_pad + m) * d;
+  est_q[dst + f] = y1;
+  est_q[dst + f + hd] = y2;
+}
+
+}  // namespace q1m

@@ -1,0 +1,77 @@
+"""The C-ABI library loads, exports every entry point include/q1m.h declares, and rejects bad
+arguments on the host before touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_prefill_dca_b200 import build, q1m
+from synth import configs as C
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "q1m.h")
+
+
+def declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(q1m_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return q1m.library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared()
+    assert len(names) >= 18
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(q1m.SIGNATURES), set(names) ^ set(q1m.SIGNATURES)
+
+
+def test_version(lib):
+    assert "sm_100a" in q1m.version()
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("dca_chunk", 1000, -2),         # c - w not a multiple of 128
+    ("local_window", -1, -1),
+    ("prefill_chunk", 100, -1),
+    ("vs_force_local", 0, -1),       # sparse needs the diagonal kept
+    ("vs_last_q", 65, -1),
+    ("in_dtype", 7, -1),
+])
+def test_invalid_params_rejected_without_launch(lib, field, value, code):
+    p = q1m.params(C.SMALL_SPARSE)
+    setattr(p, field, value)
+    w = C.SMALL_SPARSE
+    st = lib.q1m_dca_sparse_prefill(1, 1, 1, 1, None, w.seq_len, w.n_q_heads, w.n_kv_heads,
+                                    w.head_dim, ctypes.byref(p), 256, 1 << 40, None)
+    assert st == code, (st, lib.q1m_last_error())
+    assert lib.q1m_last_error().decode()
+
+
+def test_bad_shapes_rejected(lib):
+    w = C.SMALL_SPARSE
+    p = q1m.params(w)
+    assert lib.q1m_workspace_bytes(w.seq_len, 6, 4, 128, ctypes.byref(p)) == 0     # 6 % 4
+    assert lib.q1m_workspace_bytes(w.seq_len, 4, 2, 96, ctypes.byref(p)) == 0      # head_dim
+    assert lib.q1m_workspace_bytes(0, 4, 2, 128, ctypes.byref(p)) == 0
+    st = lib.q1m_dca_sparse_prefill(None, 1, 1, 1, None, w.seq_len, 4, 2, 128, ctypes.byref(p),
+                                    256, 1 << 40, None)
+    assert st == -1
+    st = lib.q1m_dca_sparse_prefill(1, 1, 1, 1, None, w.seq_len, 4, 2, 128, ctypes.byref(p),
+                                    256, 10, None)
+    assert st == -3          # workspace too small
+    st = lib.q1m_dca_sparse_prefill(1, 1, 1, 1, None, w.seq_len, 16, 2, 128, ctypes.byref(p),
+                                    256, 1 << 40, None)
+    assert st == -2          # 8 Q heads per KV head exceeds the estimator
+
+
+def test_workspace_sizes_monotone(lib):
+    small = q1m.workspace_bytes(C.L7B_128K.seq_len, 28, 4, 128, q1m.params(C.L7B_128K))
+    big = q1m.workspace_bytes(C.L7B_1M.seq_len, 28, 4, 128, q1m.params(C.L7B_1M))
+    assert 0 < small < big < 40 * 2**30
