@@ -217,6 +217,36 @@ const char* q1m_last_error(void);
 /* Library version string. */
 const char* q1m_version(void);
 
+/* ---------------------------------------------------------------------------------------
+ * Measurement
+ * ------------------------------------------------------------------------------------- */
+
+/* Stages timed by the per-stage event timers of q1m_dca_sparse_prefill. */
+enum {
+  Q1M_STAGE_TABLE = 0,     /* RoPE table                              */
+  Q1M_STAGE_KEYS = 1,      /* DCA key rotation                        */
+  Q1M_STAGE_QUERIES = 2,   /* DCA query views                         */
+  Q1M_STAGE_ESTIMATE = 3,  /* vertical-slash estimator                */
+  Q1M_STAGE_SELECT = 4,    /* budget selection                        */
+  Q1M_STAGE_MASKS = 5,     /* block masks and residual columns        */
+  Q1M_STAGE_ATTN = 6,      /* block-sparse attention kernel           */
+  Q1M_STAGE_MERGE = 7,     /* LSE merge of the DCA patterns           */
+  Q1M_NUM_STAGES = 8
+};
+
+/* Enables (1) or disables (0) per-stage CUDA-event timing inside q1m_dca_sparse_prefill on
+ * this thread; enabling also clears the accumulated times. Events are recorded on the call's
+ * stream around each stage's launches. */
+q1m_status q1m_profile_enable(int on);
+
+/* Synchronizes the recorded events and writes, per stage, the accumulated milliseconds
+ * (ms[Q1M_NUM_STAGES]) and the number of timed launches of that stage's main kernel
+ * (launches[Q1M_NUM_STAGES], nullable) since the last enable. */
+q1m_status q1m_profile_read(double* ms, int64_t* launches);
+
+/* Number of kernels this library has launched in the process so far. */
+uint64_t q1m_launch_count(void);
+
 /* Sets the budget, in SM clock cycles, of the kernels' bounded waits on the current device
  * (default 2e9, about one second); 0 restores the default. */
 q1m_status q1m_set_wait_budget(uint64_t cycles);

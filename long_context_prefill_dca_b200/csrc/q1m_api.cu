@@ -8,8 +8,10 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "q1m_device.cuh"
 #include "rope_dca.cuh"
@@ -41,8 +43,11 @@ q1m_status fail(q1m_status s, const char* fmt, ...) {
       return fail(Q1M_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(err_));     \
   } while (0)
 
+std::atomic<uint64_t> g_launches{0};
+
 #define Q1M_LAUNCHED()                                                                 \
   do {                                                                                 \
+    g_launches.fetch_add(1, std::memory_order_relaxed);                                \
     cudaError_t err_ = cudaGetLastError();                                             \
     if (err_ != cudaSuccess)                                                           \
       return fail(Q1M_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(err_)); \
@@ -53,6 +58,42 @@ q1m_status fail(q1m_status s, const char* fmt, ...) {
     q1m_status st_ = (expr);                \
     if (st_ != Q1M_OK) return st_;          \
   } while (0)
+
+// ---- per-stage event timers (opt-in, per thread) -------------------------------------------
+struct ProfRec {
+  int stage;
+  cudaEvent_t a, b;
+};
+struct StageTimer {
+  bool on = false;
+  std::vector<cudaEvent_t> pool;   // events are reused across reads
+  size_t used = 0;
+  std::vector<ProfRec> recs;
+};
+thread_local StageTimer t_prof;
+
+cudaEvent_t prof_event() {
+  if (t_prof.used == t_prof.pool.size()) {
+    cudaEvent_t ev;
+    if (cudaEventCreate(&ev) != cudaSuccess) return nullptr;
+    t_prof.pool.push_back(ev);
+  }
+  return t_prof.pool[t_prof.used++];
+}
+
+// Opens a timed interval of `stage` on stream `st`; returns its index (-1: timing off).
+int prof_begin(int stage, cudaStream_t st) {
+  if (!t_prof.on) return -1;
+  cudaEvent_t a = prof_event(), b = prof_event();
+  if (!a || !b) return -1;
+  cudaEventRecord(a, st);
+  t_prof.recs.push_back(ProfRec{stage, a, b});
+  return (int)t_prof.recs.size() - 1;
+}
+
+void prof_end(int idx, cudaStream_t st) {
+  if (idx >= 0) cudaEventRecord(t_prof.recs[idx].b, st);
+}
 
 inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 inline size_t align_up(size_t x) { return (x + 1023) & ~size_t(1023); }
@@ -354,7 +395,9 @@ q1m_status run_attn_d(const uint16_t* qv, int64_t ld_rows, const uint16_t* k_rot
   Q1M_CUDA(cudaFuncSetAttribute(block_sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const int64_t items_max = (int64_t)U * hq;
   const int grid = (int)(items_max < dev.sms ? items_max : dev.sms);
+  const int pr = prof_begin(Q1M_STAGE_ATTN, st);
   block_sparse_attn_kernel<D><<<grid, K3_THREADS, smem, st>>>(mq, mk, mv, a);
+  prof_end(pr, st);
   Q1M_LAUNCHED();
   return Q1M_OK;
 }
@@ -536,7 +579,9 @@ q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, v
   float* lse_part = at<float>(ws, L.lse_part);
   int32_t* units = at<int32_t>(ws, L.units);
   const int64_t Ld = p->dca_chunk - p->local_window;
+  int pr = prof_begin(Q1M_STAGE_TABLE, st);
   Q1M_TRY(run_rope_table(table, p->dca_chunk, d, p->rope_base, st));
+  prof_end(pr, st);
   if (L.ld_tokens > n) {
     // zero the padded key rows once so tiles past the end read finite values
     for (int g = 0; g < hkv; ++g) {
@@ -546,8 +591,12 @@ q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, v
   }
   for (int64_t s0 = 0; s0 < n; s0 += p->prefill_chunk) {
     const int64_t e = s0 + p->prefill_chunk < n ? s0 + p->prefill_chunk : n;
+    pr = prof_begin(Q1M_STAGE_KEYS, st);
     Q1M_TRY(run_rope_keys(k, v, s0, e, hkv, d, p, table, k_rot, v16, L.ld_tokens, st));
+    prof_end(pr, st);
+    pr = prof_begin(Q1M_STAGE_QUERIES, st);
     Q1M_TRY(run_rope_queries(q, s0, e, hq, d, p, table, qv, L.ld_rows, st));
+    prof_end(pr, st);
     const uint32_t* mask = nullptr;
     const int32_t *resid = nullptr, *cnt = nullptr;
     if (sparse(p)) {
@@ -555,17 +604,25 @@ q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, v
       float* slash = at<float>(ws, L.slash);
       int32_t* V = at<int32_t>(ws, L.V);
       int32_t* Sx = at<int32_t>(ws, L.Sx);
+      pr = prof_begin(Q1M_STAGE_ESTIMATE, st);
       if (d == 128) Q1M_TRY(run_estimate_d<128>(q, k_rot, L.ld_tokens, s0, e, hq, hkv, p, table, vert, slash, L.ld_tokens, at<void>(ws, L.est), dev, st));
       else Q1M_TRY(run_estimate_d<64>(q, k_rot, L.ld_tokens, s0, e, hq, hkv, p, table, vert, slash, L.ld_tokens, at<void>(ws, L.est), dev, st));
+      prof_end(pr, st);
+      pr = prof_begin(Q1M_STAGE_SELECT, st);
       Q1M_TRY(run_select(vert, slash, L.ld_tokens, e, hq, p, V, Sx, st));
+      prof_end(pr, st);
+      pr = prof_begin(Q1M_STAGE_MASKS, st);
       Q1M_TRY(run_masks(V, Sx, s0, e, hq, p, at<uint32_t>(ws, L.mask), at<int32_t>(ws, L.resid), at<int32_t>(ws, L.cnt), st));
+      prof_end(pr, st);
       mask = at<uint32_t>(ws, L.mask);
       resid = at<int32_t>(ws, L.resid);
       cnt = at<int32_t>(ws, L.cnt);
     }
     if (d == 128) Q1M_TRY(run_attn_d<128>(qv, L.ld_rows, k_rot, v16, L.ld_tokens, mask, resid, cnt, s0, e, hq, hkv, p, o_part, lse_part, units, dev, st));
     else Q1M_TRY(run_attn_d<64>(qv, L.ld_rows, k_rot, v16, L.ld_tokens, mask, resid, cnt, s0, e, hq, hkv, p, o_part, lse_part, units, dev, st));
+    pr = prof_begin(Q1M_STAGE_MERGE, st);
     Q1M_TRY(run_merge(o_part, lse_part, 3, L.ld_rows, s0, e, n, hq, d, p->out_dtype, Ld, out, lse, st));
+    prof_end(pr, st);
   }
   return Q1M_OK;
 }
@@ -608,6 +665,30 @@ q1m_status q1m_status_poll(void* stream) {
   }
   return Q1M_OK;
 }
+
+q1m_status q1m_profile_enable(int on) {
+  t_prof.on = on != 0;
+  t_prof.used = 0;
+  t_prof.recs.clear();
+  return Q1M_OK;
+}
+
+q1m_status q1m_profile_read(double* ms, int64_t* launches) {
+  if (!ms) return fail(Q1M_ERR_INVALID, "ms is NULL");
+  for (int i = 0; i < Q1M_NUM_STAGES; ++i) { ms[i] = 0.0; if (launches) launches[i] = 0; }
+  for (const ProfRec& r : t_prof.recs) {
+    Q1M_CUDA(cudaEventSynchronize(r.b));
+    float t = 0.f;
+    Q1M_CUDA(cudaEventElapsedTime(&t, r.a, r.b));
+    ms[r.stage] += t;
+    if (launches) launches[r.stage] += 1;
+  }
+  t_prof.used = 0;
+  t_prof.recs.clear();
+  return Q1M_OK;
+}
+
+uint64_t q1m_launch_count(void) { return g_launches.load(); }
 
 q1m_status q1m_set_wait_budget(uint64_t cycles) {
   unsigned long long v = cycles ? (unsigned long long)cycles : 2000000000ull;

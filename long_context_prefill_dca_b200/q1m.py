@@ -64,6 +64,9 @@ SIGNATURES = {
     "q1m_last_error": (ctypes.c_char_p, []),
     "q1m_version": (ctypes.c_char_p, []),
     "q1m_set_wait_budget": (c_int, [c_u64]),
+    "q1m_profile_enable": (c_int, [c_int]),
+    "q1m_profile_read": (c_int, [ctypes.POINTER(c_dbl), ctypes.POINTER(c_i64)]),
+    "q1m_launch_count": (c_u64, []),
     "q1m_selftest_wait_timeout": (c_int, [c_u64, c_vp]),
 }
 
@@ -215,6 +218,25 @@ def set_wait_budget(cycles: int) -> None:
 
 def selftest_wait_timeout(cycles: int, stream=None) -> int:
     return library().q1m_selftest_wait_timeout(cycles, stream_handle(stream))
+
+
+STAGES = ["table", "keys", "queries", "estimate", "select", "masks", "attn", "merge"]
+
+
+def profile_enable(on: bool = True) -> None:
+    _call("q1m_profile_enable", 1 if on else 0)
+
+
+def profile_read() -> dict:
+    """{stage: (ms, launches)} accumulated since profile_enable()."""
+    ms = (c_dbl * len(STAGES))()
+    n = (c_i64 * len(STAGES))()
+    _call("q1m_profile_read", ms, n)
+    return {name: (ms[i], n[i]) for i, name in enumerate(STAGES)}
+
+
+def launch_count() -> int:
+    return int(library().q1m_launch_count())
 
 
 def version() -> str:
