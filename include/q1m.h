@@ -190,6 +190,31 @@ q1m_status q1m_block_sparse_attn(const uint16_t* qv, int64_t ld_rows, const uint
                                  const q1m_params* p, float* o_part, float* lse_part,
                                  void* scratch, size_t scratch_bytes, void* stream);
 
+/* Allocation-free variant of q1m_block_sparse_attn, for callers that cannot call cudaMalloc
+ * and cannot hand the library a scratch buffer: for example code that runs under a strict
+ * memory planner or pool that owns every device allocation, or a host thread on a latency
+ * path that must never wait on the allocator. The pages have no counterpart to this entry
+ * point; it exists only for such callers.
+ * Same arguments and results as q1m_block_sparse_attn, without scratch: the work-unit list
+ * lives in a static device array of Q1M_NOALLOC_UNITS int32 (64 KiB) that every GPU which
+ * loads the library holds until the process exits. A chunk may therefore have at most
+ * Q1M_NOALLOC_MAX_QUERY_BLOCKS query blocks of 128 rows (1,397,248 rows); larger chunks are
+ * rejected with Q1M_ERR_UNSUPPORTED before anything is launched. The call allocates nothing
+ * (no cudaMalloc, cudaFree or allocating library routine). The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress) with that device current, so
+ * make that first call before any stream capture. All calls share the one array, and each
+ * call rewrites every entry it reads; calls that can overlap on the GPU (different
+ * streams, or devices sharing it) race on it and must be serialised by the caller. */
+#define Q1M_NOALLOC_UNITS 16384
+#define Q1M_NOALLOC_MAX_QUERY_BLOCKS 10916
+q1m_status q1m_block_sparse_attn_noalloc(const uint16_t* qv, int64_t ld_rows,
+                                         const uint16_t* k_rot, const uint16_t* v16,
+                                         int64_t ld_tokens, const uint32_t* mask,
+                                         const int32_t* resid, const int32_t* cnt, int64_t s0,
+                                         int64_t e, int n_q_heads, int n_kv_heads, int head_dim,
+                                         const q1m_params* p, float* o_part, float* lse_part,
+                                         void* stream);
+
 /* Log-sum-exp merge of the DCA patterns' partial results for rows [s0, e)
  * (lse = log2 sum_x 2^lse_x, out = sum_x 2^(lse_x - lse) o_x):
  * out[i][h][:] in out_dtype ([N][Hq][D] layout) and lse[h][i] (natural log, nullable).

@@ -719,3 +719,52 @@ extern "C" q1m_status q1m_selftest_wait_timeout(uint64_t cycles, void* stream) {
   Q1M_TRY(q1m_set_wait_budget(0));
   return st;
 }
+
+// =============================================================================================
+// Allocation-free attention entry point: the work-unit list in a static device array.
+// =============================================================================================
+namespace {
+static __device__ __align__(256) int32_t g_noalloc_units[Q1M_NOALLOC_UNITS];
+std::mutex g_noalloc_mu;
+constexpr int kMaxDevices = 64;
+int32_t* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_units on the current device (looked up once per device; the
+// array's name in host code is only a stand-in for the symbol).
+q1m_status noalloc_units(int32_t** out) {
+  int dev = 0;
+  Q1M_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(Q1M_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    Q1M_CUDA(cudaGetSymbolAddress(&ptr, g_noalloc_units));
+    g_noalloc_ptr[dev] = static_cast<int32_t*>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return Q1M_OK;
+}
+}  // namespace
+
+extern "C" q1m_status q1m_block_sparse_attn_noalloc(
+    const uint16_t* qv, int64_t ld_rows, const uint16_t* k_rot, const uint16_t* v16,
+    int64_t ld_tokens, const uint32_t* mask, const int32_t* resid, const int32_t* cnt, int64_t s0,
+    int64_t e, int hq, int hkv, int d, const q1m_params* p, float* o_part, float* lse_part,
+    void* stream) {
+  Q1M_TRY(check_shape(e > 0 ? e : 1, hq, hkv, d, p));
+  if (!qv || !k_rot || !v16 || !o_part || !lse_part) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (mask && (!cnt || (p->vs_vertical > 0 && !resid))) return fail(Q1M_ERR_INVALID, "mask without counts/residuals");
+  if (s0 < 0 || e <= s0 || s0 % 128 || ld_rows < e - s0 || ld_rows % 128 || ld_tokens < e || ld_tokens % 128)
+    return fail(Q1M_ERR_INVALID, "bad range");
+  const int64_t nqb = (e - s0 + 127) / 128;
+  if (nqb > Q1M_NOALLOC_MAX_QUERY_BLOCKS ||
+      q1m_attn_scratch_bytes(s0, e, hq, d) > sizeof(int32_t) * Q1M_NOALLOC_UNITS)
+    return fail(Q1M_ERR_UNSUPPORTED, "chunk of %lld query blocks exceeds the static work list (%d blocks)",
+                (long long)nqb, Q1M_NOALLOC_MAX_QUERY_BLOCKS);
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  int32_t* units = nullptr;
+  Q1M_TRY(noalloc_units(&units));
+  if (d == 128) return run_attn_d<128>(qv, ld_rows, k_rot, v16, ld_tokens, mask, resid, cnt, s0, e, hq, hkv, p, o_part, lse_part, units, dev, S(stream));
+  return run_attn_d<64>(qv, ld_rows, k_rot, v16, ld_tokens, mask, resid, cnt, s0, e, hq, hkv, p, o_part, lse_part, units, dev, S(stream));
+}

@@ -58,6 +58,9 @@ SIGNATURES = {
     "q1m_block_sparse_attn": (c_int, [c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_i64,
                                       c_i64, c_int, c_int, c_int, PP, c_vp, c_vp, c_vp, c_size,
                                       c_vp]),
+    "q1m_block_sparse_attn_noalloc": (c_int, [c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp,
+                                              c_i64, c_i64, c_int, c_int, c_int, PP, c_vp, c_vp,
+                                              c_vp]),
     "q1m_lse_merge": (c_int, [c_vp, c_vp, c_int, c_i64, c_i64, c_i64, c_i64, c_int, c_int, c_int,
                               PP, c_vp, c_vp, c_vp]),
     "q1m_status_poll": (c_int, [c_vp]),
@@ -193,6 +196,13 @@ def block_sparse_attn(qv, ld_rows, k_rot, v16, ld_tokens, mask, resid, cnt, s0, 
     _call("q1m_block_sparse_attn", ptr(qv), ld_rows, ptr(k_rot), ptr(v16), ld_tokens, ptr(mask),
           ptr(resid), ptr(cnt), s0, e, hq, hkv, d, ctypes.byref(p), ptr(o_part), ptr(lse_part),
           ptr(scratch), scratch_bytes, stream_handle(stream))
+
+
+def block_sparse_attn_noalloc(qv, ld_rows, k_rot, v16, ld_tokens, mask, resid, cnt, s0, e, hq,
+                              hkv, d, p: Params, o_part, lse_part, stream=None):
+    _call("q1m_block_sparse_attn_noalloc", ptr(qv), ld_rows, ptr(k_rot), ptr(v16), ld_tokens,
+          ptr(mask), ptr(resid), ptr(cnt), s0, e, hq, hkv, d, ctypes.byref(p), ptr(o_part),
+          ptr(lse_part), stream_handle(stream))
 
 
 def lse_merge(o_part, lse_part, n_parts, ld_rows, s0, e, n, hq, d, out_dtype, p, out, lse,
