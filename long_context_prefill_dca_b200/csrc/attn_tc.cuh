@@ -16,7 +16,8 @@
 //    (Toeplitz block masks) they mostly do.
 //  * Warp roles: warps 0-3 softmax of slot 0, warps 4-7 softmax of slot 1, warp 8 loads
 //    (TMA for key blocks, cp.async gathers for residual vertical columns), warp 9 issues
-//    tcgen05.mma and owns tensor memory.
+//    tcgen05.mma and owns tensor memory, warps 10-11 idle; the softmax warpgroups take
+//    registers from the third warpgroup (setmaxnreg) to hold a whole S row.
 //  * Tensor memory per slot: S (128 fp32 columns), O (D fp32 columns); the softmax writes
 //    P as packed fp16 over the first 64 columns of S and the PV product reads it from
 //    tensor memory (A operand), with V as an MN-major shared-memory operand.
@@ -32,7 +33,10 @@ namespace q1m {
 
 constexpr int K3_NK = 2;        // K stages
 constexpr int K3_NV = 2;        // V stages
-constexpr int K3_THREADS = 320;
+constexpr int K3_THREADS = 384;   // 3 warpgroups: softmax slot 0, softmax slot 1, loader + MMA
+// register split (setmaxnreg): launch 384 x 168 = 64,512; 2 x 128 x 208 + 128 x 88 = 64,512
+constexpr int K3_REGS_SOFTMAX = 208;
+constexpr int K3_REGS_OTHER = 88;
 constexpr float K3_RESCALE_THRESHOLD = 8.0f;
 
 struct K3Args {
@@ -243,146 +247,163 @@ __device__ void k3_producer(K3Smem<D>& sm, const K3Args& a, const CUtensorMap* m
 }
 
 // --------------------------------------------------------------------------------------
-// MMA warp (one thread issues)
+// MMA warp (one thread issues). Per-slot state lives in registers (static slot indices).
 // --------------------------------------------------------------------------------------
+struct K3Slot {
+  int pend_v = -1;            // V stage of the slot's pending PV (-1: none)
+  uint32_t pend_kt = 0;       // tile index of that PV
+  bool pend_last = false;     // it is the slot's last tile of the item
+  bool o_started = false;     // O holds a partial sum of the current item
+  uint32_t qn = 0, pn = 0, pvd_issued = 0, pvd_waited = 0;
+};
+
+// PV of the slot's pending tile: O (+)= P V, P read from tensor memory.
+template <int D, int S>
+__device__ __forceinline__ bool k3_pv(K3Smem<D>& sm, K3Slot& sl, uint32_t tb, uint32_t& v_users) {
+  constexpr uint32_t IDESC_PV = idesc_f16(128, D, 1);
+  if (!mbar_wait(&sm.p_full[S], sl.pn & 1)) return false;
+  ++sl.pn;
+  const int vst = sl.pend_v;
+  if (!mbar_wait(&sm.v_full[vst], (sl.pend_kt / K3_NV) & 1)) return false;
+  tc_fence_after();
+  const uint32_t o_t = tb + 256u * S + 128u, p_t = tb + 256u * S;
+  const uint32_t vbase = smem_u32(sm.v[vst]);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ts(o_t, p_t + kk * 8u, sdesc_sw128(vbase + kk * 2048u, 16384u, 1024u), IDESC_PV,
+           (sl.o_started || kk > 0) ? 1u : 0u);
+  sl.o_started = true;
+  // P lives in S's columns: the slot's next QK^T may overwrite them only after this PV read them
+  mma_commit(&sm.pv_done[S]);
+  ++sl.pvd_issued;
+  if (sl.pend_last) { mma_commit(&sm.o_done[S]); sl.o_started = false; }
+  const uint32_t sh = 4u * (uint32_t)vst;
+  const uint32_t u = ((v_users >> sh) & 0xFu) - 1u;
+  v_users = (v_users & ~(0xFu << sh)) | (u << sh);
+  if (u == 0) mma_commit(&sm.v_empty[vst]);
+  sl.pend_v = -1;
+  return true;
+}
+
+// S = Q K^T for the slot on K stage kst.
+template <int D, int S>
+__device__ __forceinline__ bool k3_qk(K3Smem<D>& sm, K3Slot& sl, int& rem, bool& first, int kst,
+                                      int vst, uint32_t kt, int diag, int ncols, uint32_t tb) {
+  constexpr uint32_t IDESC_QK = idesc_f16(128, 128, 0);
+  if (first) {
+    if (!mbar_wait(&sm.q_full[S], sl.qn & 1)) return false;
+    ++sl.qn;
+    first = false;
+    tc_fence_after();
+  }
+  if (sl.pvd_waited < sl.pvd_issued) {
+    if (!mbar_wait(&sm.pv_done[S], sl.pvd_waited & 1)) return false;
+    ++sl.pvd_waited;
+  }
+  --rem;
+  const bool last = rem == 0;
+  sm.meta[S] = ((diag >> S) & 1) | (ncols << 8) | ((int)last << 16);
+  mbar_arrive(&sm.s_full[S]);
+  const uint32_t s_t = tb + 256u * S;
+  const uint32_t qbase = smem_u32(sm.q[S]), kbase = smem_u32(sm.k[kst]);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
+    mma_ss(s_t, sdesc_sw128(qbase + off, 16u, 1024u), sdesc_sw128(kbase + off, 16u, 1024u),
+           IDESC_QK, kk > 0 ? 1u : 0u);
+  }
+  mma_commit(&sm.s_full[S]);
+  if (last) mma_commit(&sm.q_empty[S]);
+  sl.pend_v = vst;
+  sl.pend_kt = kt;
+  sl.pend_last = last;
+  return true;
+}
+
 template <int D>
 __device__ void k3_mma(K3Smem<D>& sm, const K3Args& a, int nitems) {
-  constexpr uint32_t IDESC_QK = idesc_f16(128, 128, 0);
-  constexpr uint32_t IDESC_PV = idesc_f16(128, D, 1);
   const uint32_t tb = sm.tmem_base;
   uint32_t kt = 0;
-  uint32_t qn[2] = {0, 0}, sn[2] = {0, 0}, pn[2] = {0, 0};
-  int pend_v[2] = {-1, -1};     // V stage of the slot's pending PV (-1: none)
-  uint32_t pend_kt[2] = {0, 0};
-  bool pend_last[2] = {false, false};
-  bool o_started[2] = {false, false};
-  uint32_t pvd_issued[2] = {0, 0}, pvd_waited[2] = {0, 0};
-  int v_users[K3_NV] = {};
+  K3Slot s0, s1;
+  uint32_t v_users = 0;       // 4 bits per V stage: PVs still to issue on it
   bool ok = true;
-
-  auto issue_pv = [&](int s) -> bool {
-    if (!mbar_wait(&sm.p_full[s], pn[s] & 1)) return false;
-    ++pn[s];
-    const int vst = pend_v[s];
-    if (!mbar_wait(&sm.v_full[vst], (pend_kt[s] / K3_NV) & 1)) return false;
-    tc_fence_after();
-    const uint32_t o_t = tb + 256u * s + 128u, p_t = tb + 256u * s;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t vb = smem_u32(sm.v[vst]) + kk * 2048u;
-      mma_ts(o_t, p_t + kk * 8u, sdesc_sw128(vb, 16384u, 1024u), IDESC_PV,
-             (o_started[s] || kk > 0) ? 1u : 0u);
-    }
-    o_started[s] = true;
-    // P lives in S's columns: the next QK^T of this slot may overwrite them only after
-    // this PV has read them
-    mma_commit(&sm.pv_done[s]);
-    ++pvd_issued[s];
-    if (pend_last[s]) { mma_commit(&sm.o_done[s]); o_started[s] = false; }
-    if (--v_users[vst] == 0) mma_commit(&sm.v_empty[vst]);
-    pend_v[s] = -1;
-    return true;
-  };
-
   for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
     const K3Item I = k3_item(a, it);
-    int rem[2] = {I.ntiles[0], I.ntiles[1]};
-    bool first[2] = {true, true};
-    while ((rem[0] > 0 || rem[1] > 0) && ok) {
+    int rem0 = I.ntiles[0], rem1 = I.ntiles[1];
+    bool first0 = true, first1 = true;
+    while ((rem0 > 0 || rem1 > 0) && ok) {
       const int kst = kt % K3_NK, vst = kt % K3_NV;
       ok = mbar_wait(&sm.k_full[kst], (kt / K3_NK) & 1);
       if (!ok) break;
       tc_fence_after();
       const int flags = sm.desc[kst][0], diag = sm.desc[kst][1], ncols = sm.desc[kst][2];
-      int users = 0;
-      for (int s = 0; s < 2 && ok; ++s) {
-        if (pend_v[s] >= 0) { ok = issue_pv(s); if (!ok) break; }
-        if (!(flags & (1 << s))) continue;
-        if (first[s]) {
-          ok = mbar_wait(&sm.q_full[s], qn[s] & 1);
-          if (!ok) break;
-          ++qn[s];
-          first[s] = false;
-          tc_fence_after();
-        }
-        if (pvd_waited[s] < pvd_issued[s]) {
-          ok = mbar_wait(&sm.pv_done[s], pvd_waited[s] & 1);
-          if (!ok) break;
-          ++pvd_waited[s];
-        }
-        --rem[s];
-        const bool last = rem[s] == 0;
-        sm.meta[s] = ((diag >> s) & 1) | (ncols << 8) | ((int)last << 16);
-        mbar_arrive(&sm.s_full[s]);
-        const uint32_t s_t = tb + 256u * s;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
-          mma_ss(s_t, sdesc_sw128(smem_u32(sm.q[s]) + off, 16u, 1024u),
-                 sdesc_sw128(smem_u32(sm.k[kst]) + off, 16u, 1024u), IDESC_QK, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&sm.s_full[s]);
-        ++sn[s];
-        if (last) mma_commit(&sm.q_empty[s]);
-        pend_v[s] = vst;
-        pend_kt[s] = kt;
-        pend_last[s] = last;
-        ++users;
-      }
+      uint32_t users = 0;
+      if (ok && s0.pend_v >= 0) ok = k3_pv<D, 0>(sm, s0, tb, v_users);
+      if (ok && (flags & 1)) { ok = k3_qk<D, 0>(sm, s0, rem0, first0, kst, vst, kt, diag, ncols, tb); ++users; }
+      if (ok && s1.pend_v >= 0) ok = k3_pv<D, 1>(sm, s1, tb, v_users);
+      if (ok && (flags & 2)) { ok = k3_qk<D, 1>(sm, s1, rem1, first1, kst, vst, kt, diag, ncols, tb); ++users; }
       if (!ok) break;
-      v_users[vst] = users;
+      const uint32_t sh = 4u * (uint32_t)vst;
+      v_users = (v_users & ~(0xFu << sh)) | (users << sh);
       mma_commit(&sm.k_empty[kst]);
       ++kt;
     }
   }
-  for (int s = 0; s < 2 && ok; ++s)
-    if (pend_v[s] >= 0) ok = issue_pv(s);
+  if (ok && s0.pend_v >= 0) ok = k3_pv<D, 0>(sm, s0, tb, v_users);
+  if (ok && s1.pend_v >= 0) ok = k3_pv<D, 1>(sm, s1, tb, v_users);
   mma_commit(&sm.drain);
   mbar_wait(&sm.drain, 0);
 }
 
 // --------------------------------------------------------------------------------------
-// Softmax warpgroup of one slot: thread t owns row t of the slot's query block.
+// Softmax warpgroup of slot S: thread t owns row t of the slot's query block.
 // --------------------------------------------------------------------------------------
-template <int D>
-__device__ void k3_softmax(K3Smem<D>& sm, const K3Args& a, int nitems, int s) {
-  const int t = threadIdx.x - 128 * s;          // row within the query block
+template <int D, int S>
+__device__ void k3_softmax(K3Smem<D>& sm, const K3Args& a, int nitems) {
+  const int t = threadIdx.x - 128 * S;          // row within the query block
   const uint32_t wq = warp_id() & 3u;           // TMEM lane quarter of this warp
-  const uint32_t tb = sm.tmem_base + ((32u * wq) << 16) + 256u * s;
+  const uint32_t tb = sm.tmem_base + ((32u * wq) << 16) + 256u * S;
   uint32_t sn = 0, on = 0;
   bool ok = true;
   for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
     const K3Item I = k3_item(a, it);
-    if (!I.valid[s]) continue;
-    const int64_t row = I.B[s] * 128 + t;       // global row
+    if (!I.valid[S]) continue;
+    const int64_t row = I.B[S] * 128 + t;       // global row
     const int64_t rl = row - a.s0;              // row within the chunk
     const bool live = row < a.e;
     float* lse_out = a.lse_part + ((int64_t)I.x * a.hq + I.h) * a.ld_rows + rl;
-    if (I.ntiles[s] == 0) {
+    if (I.ntiles[S] == 0) {
       if (live) *lse_out = -INFINITY;
       continue;
     }
     float m = -INFINITY, l = 0.f;
     bool o_valid = false;
-    for (int tt = 0; tt < I.ntiles[s]; ++tt) {
-      ok = mbar_wait_warp(&sm.s_full[s], sn & 1);
+    for (int tt = 0; tt < I.ntiles[S]; ++tt) {
+      ok = mbar_wait_warp(&sm.s_full[S], sn & 1);
       if (!ok) break;
       ++sn;
       tc_fence_after();
-      const int meta = sm.meta[s];
+      const int meta = sm.meta[S];
       const bool diag = meta & 1;
       const int ncols = (meta >> 8) & 0xFF;
-      float x[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tb + 32u * c, reinterpret_cast<uint32_t*>(x) + 32 * c);
+      // the whole 128-column S row in registers: one tensor-memory load and wait per tile
+      uint32_t xr[128];
+      tmem_ld128(tb, xr);
+      float* x = reinterpret_cast<float*>(xr);
       if (diag || ncols < 128) {
         const int lim = diag ? t : ncols - 1;
 #pragma unroll
         for (int c = 0; c < 128; ++c) if (c > lim) x[c] = -INFINITY;
       }
-      float mx = x[0];
+      // row maximum: eight independent chains of 3-input max
+      float a8[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      for (int k = 0; k < 8; ++k) a8[k] = x[k];
+#pragma unroll
+      for (int c = 8; c < 128; c += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a8[k] = fmax3(a8[k], x[c + k], x[c + 8 + k]);
+      const float mx = fmaxf(fmax3(a8[0], a8[1], a8[2]), fmax3(fmax3(a8[3], a8[4], a8[5]), a8[6], a8[7]));
       const bool need = mx > m + K3_RESCALE_THRESHOLD;
       if (__any_sync(0xFFFFFFFFu, need)) {
         const float m_new = need ? mx : m;
@@ -401,24 +422,35 @@ __device__ void k3_softmax(K3Smem<D>& sm, const K3Args& a, int nitems, int s) {
         m = m_new;
       }
       const float mu = m == -INFINITY ? 0.f : m;
-      uint32_t pk[64];
-      float sum = 0.f;
+      // p = 2^(x - mu) in packed pairs, four independent packed sums; P goes to tensor
+      // memory 32 keys (16 packed words) at a time
+      const uint64_t nmu = f2_pack(-mu, -mu);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2(x[2 * c] - mu), p1 = ex2(x[2 * c + 1] - mu);
-        sum += p0 + p1;
-        pk[c] = pack_f16x2(p0, p1);
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int j = 32 * ch + 2 * c;
+          float d0, d1;
+          f2_unpack(f2_add(f2_pack(x[j], x[j + 1]), nmu), d0, d1);
+          const float p0 = ex2(d0), p1 = ex2(d1);
+          acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
+          pk[c] = pack_f16x2(p0, p1);
+        }
+        tmem_st16(tb + 16u * ch, pk);
       }
-      l += sum;
-      tmem_st32(tb, pk);
-      tmem_st32(tb + 32u, pk + 32);
+      float s0, s1, s2, s3;
+      f2_unpack(f2_add(acc[0], acc[1]), s0, s1);
+      f2_unpack(f2_add(acc[2], acc[3]), s2, s3);
+      l += (s0 + s1) + (s2 + s3);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full[s]);
+      mbar_arrive(&sm.p_full[S]);
       o_valid = true;
     }
     if (!ok) break;
-    ok = mbar_wait_warp(&sm.o_done[s], on & 1);
+    ok = mbar_wait_warp(&sm.o_done[S], on & 1);
     if (!ok) break;
     ++on;
     tc_fence_after();
@@ -466,9 +498,15 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_co
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (w < 8) k3_softmax<D>(sm, a, nitems, w >> 2);
-  else if (w == 8) k3_producer<D>(sm, a, &mq, &mk, &mv, nitems);
-  else if (lane_id() == 0) k3_mma<D>(sm, a, nitems);
+  if (w < 8) {
+    regs_increase<K3_REGS_SOFTMAX>();
+    if (w < 4) k3_softmax<D, 0>(sm, a, nitems);
+    else k3_softmax<D, 1>(sm, a, nitems);
+  } else {
+    regs_decrease<K3_REGS_OTHER>();
+    if (w == 8) k3_producer<D>(sm, a, &mq, &mk, &mv, nitems);
+    else if (w == 9 && lane_id() == 0) k3_mma<D>(sm, a, nitems);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
