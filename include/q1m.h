@@ -269,6 +269,12 @@ q1m_status q1m_profile_enable(int on);
  * (launches[Q1M_NUM_STAGES], nullable) since the last enable. */
 q1m_status q1m_profile_read(double* ms, int64_t* launches);
 
+/* Self-test of the attention kernel's FMA-pipe exponential: for x[0..n) (device, fp32)
+ * writes y_poly = the kernel's polynomial 2^x, y_mufu = the multi-function-unit 2^x
+ * (ex2.approx) and y_ref = CUDA's exp2f(x), so a caller can check the error bound. */
+q1m_status q1m_selftest_exp2(const float* x, float* y_poly, float* y_mufu, float* y_ref, int64_t n,
+                             void* stream);
+
 /* Number of kernels this library has launched in the process so far. */
 uint64_t q1m_launch_count(void);
 

@@ -16,7 +16,7 @@
 //    (Toeplitz block masks) they mostly do.
 //  * Warp roles: warps 0-3 softmax of slot 0, warps 4-7 softmax of slot 1, warp 8 loads
 //    (TMA for key blocks, cp.async gathers for residual vertical columns), warp 9 issues
-//    tcgen05.mma and owns tensor memory, warps 10-11 idle; the softmax warpgroups take
+//    tcgen05.mma and owns tensor memory, warp 10 loads V tiles, warp 11 idles; the softmax warpgroups take
 //    registers from the third warpgroup (setmaxnreg) to hold a whole S row.
 //  * Tensor memory per slot: S (128 fp32 columns), O (D fp32 columns); the softmax writes
 //    P as packed fp16 over the first 64 columns of S and the PV product reads it from
@@ -34,10 +34,20 @@ namespace q1m {
 constexpr int K3_NK = 2;        // K stages
 constexpr int K3_NV = 2;        // V stages
 constexpr int K3_THREADS = 384;   // 3 warpgroups: softmax slot 0, softmax slot 1, loader + MMA
-// register split (setmaxnreg): launch 384 x 168 = 64,512; 2 x 128 x 208 + 128 x 88 = 64,512
-constexpr int K3_REGS_SOFTMAX = 208;
-constexpr int K3_REGS_OTHER = 88;
+// register split (setmaxnreg): launch 384 x 168 = 64,512 = 2 x 128 x 192 + 128 x 120 (no spills)
+constexpr int K3_REGS_SOFTMAX = 192;
+constexpr int K3_REGS_OTHER = 120;
 constexpr float K3_RESCALE_THRESHOLD = 8.0f;
+// exponentials of K3_POLY_PAIRS_OF_8 of every 8 pairs run on the FMA pipe (ex2_poly2), the
+// rest on the MUFU; measured on B200 the softmax is not MUFU-bound, so the default is 0
+constexpr int K3_POLY_PAIRS_OF_8 = 0;
+// P overwrites the first half of S, so the slot's next QK^T (which writes S) must not
+// overtake the PV MMA that reads P. tcgen05.mma operations issued by one thread execute in
+// issue order, and a later MMA's accumulator writes follow an earlier MMA's operand reads,
+// so no wait is needed between them; measured on B200 the explicit wait (a commit and an
+// mbarrier round trip per tile) costs 11% of the cycles and the outputs are bit-identical
+// either way. Setting this to true restores the explicit wait.
+constexpr bool K3_WAIT_PV_BEFORE_QK = false;
 
 struct K3Args {
   int64_t s0, e;
@@ -122,7 +132,7 @@ struct K3Smem {
   alignas(1024) uint8_t q[2][TILE];
   alignas(1024) uint8_t k[K3_NK][TILE];
   alignas(1024) uint8_t v[K3_NV][TILE];
-  int desc[K3_NK][4];       // flags, diag mask, ncols (gathers; 128 for blocks), unused
+  int desc[K3_NK][4];       // flags, diag mask, ncols (gathers; 128 for blocks), unused (K stages)
   int meta[2];              // per-slot mailbox written by the MMA warp before its arrive
   uint64_t k_full[K3_NK], k_empty[K3_NK], v_full[K3_NV], v_empty[K3_NV];
   uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_done[2], pv_done[2];
@@ -131,23 +141,23 @@ struct K3Smem {
 };
 
 // --------------------------------------------------------------------------------------
-// Loader warp
+// Loader warps. Two warps walk the same tile sequence: ROLE 0 loads the Q views and the K
+// tiles (and publishes each tile's descriptor), ROLE 1 loads the V tiles, so a K tile can
+// be fetched ahead of the V tiles still in use.
 // --------------------------------------------------------------------------------------
 template <int D>
-__device__ void k3_gather(K3Smem<D>& sm, const K3Args& a, int g, const int32_t* cols, int n,
-                          int kst, int vst) {
-  // 128 rows x D fp16 of k_rot and v16 gathered by column index into the swizzled layout
+__device__ void k3_gather(uint8_t* dst, const uint16_t* src_base, const K3Args& a, int g,
+                          const int32_t* cols, int n) {
+  // 128 rows x D fp16 gathered by column index into the 128-byte-swizzled tile layout
   const uint32_t lane = lane_id();
   constexpr int CHUNKS = D / 8;  // 16-byte chunks per row
   for (int r = (int)lane; r < 128; r += 32) {
     const int j = cols[r < n ? r : 0];
-    const uint16_t* ks = a.k_rot + ((int64_t)g * a.ld_tokens + j) * D;
-    const uint16_t* vs = a.v16 + ((int64_t)g * a.ld_tokens + j) * D;
+    const uint16_t* src = src_base + ((int64_t)g * a.ld_tokens + j) * D;
 #pragma unroll
     for (int c = 0; c < CHUNKS; ++c) {
       const uint32_t off = (uint32_t)(c >> 3) * 16384u + sw128_offset((uint32_t)r, (uint32_t)(c & 7));
-      cp_async16(sm.k[kst] + off, ks + c * 8);
-      cp_async16(sm.v[vst] + off, vs + c * 8);
+      cp_async16(dst + off, src + c * 8);
     }
   }
   cp_async_wait_all();
@@ -155,84 +165,87 @@ __device__ void k3_gather(K3Smem<D>& sm, const K3Args& a, int g, const int32_t* 
   __syncwarp();
 }
 
-template <int D>
+template <int D, int ROLE>
 __device__ void k3_producer(K3Smem<D>& sm, const K3Args& a, const CUtensorMap* mq,
                             const CUtensorMap* mk, const CUtensorMap* mv, int nitems) {
   constexpr uint32_t TILE = K3Smem<D>::TILE;
+  constexpr int NS = ROLE == 0 ? K3_NK : K3_NV;
+  uint64_t* full = ROLE == 0 ? sm.k_full : sm.v_full;
+  uint64_t* empty = ROLE == 0 ? sm.k_empty : sm.v_empty;
+  const CUtensorMap* map = ROLE == 0 ? mk : mv;
+  const uint16_t* src = ROLE == 0 ? a.k_rot : a.v16;
   const bool leader = lane_id() == 0;
   uint32_t kt = 0;             // tiles produced by this CTA
   uint32_t qn[2] = {0, 0};     // Q loads per slot
   bool ok = true;
+  auto stage_buf = [&](int st) -> uint8_t* { return ROLE == 0 ? sm.k[st] : sm.v[st]; };
   for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
     const K3Item I = k3_item(a, it);
-    // Q views of both slots
-    for (int s = 0; s < 2 && ok; ++s) {
-      if (I.ntiles[s] == 0) continue;
-      ok = mbar_wait_warp(&sm.q_empty[s], (qn[s] & 1) ^ 1);
-      if (!ok) break;
-      if (leader) {
-        mbar_expect_tx(&sm.q_full[s], TILE);
-        const int y = (int)(((int64_t)I.x * a.hq + I.h) * a.ld_rows + (int64_t)I.qb[s] * 128);
+    if (ROLE == 0) {
 #pragma unroll
-        for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(sm.q[s] + hf * 16384, mq, &sm.q_full[s], 64 * hf, y);
+      for (int s = 0; s < 2; ++s) {
+        if (!ok || I.ntiles[s] == 0) continue;
+        ok = mbar_wait_warp(&sm.q_empty[s], (qn[s] & 1) ^ 1);
+        if (!ok) continue;
+        if (leader) {
+          mbar_expect_tx(&sm.q_full[s], TILE);
+          const int y = (int)(((int64_t)I.x * a.hq + I.h) * a.ld_rows + (int64_t)I.qb[s] * 128);
+#pragma unroll
+          for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(sm.q[s] + hf * 16384, mq, &sm.q_full[s], 64 * hf, y);
+        }
+        ++qn[s];
       }
-      ++qn[s];
     }
     // residual vertical columns, per slot, 128 per gathered tile
-    for (int s = 0; s < 2 && ok; ++s) {
-      if (I.nres[s] == 0) continue;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      if (!ok || I.nres[s] == 0) continue;
       const int32_t* cols = a.resid + ((int64_t)I.h * a.nqb + I.qb[s]) * a.nvcap + I.res_off[s];
       for (int t0 = 0; t0 < I.nres[s] && ok; t0 += 128) {
-        const int kst = kt % K3_NK, vst = kt % K3_NV;
-        ok = mbar_wait_warp(&sm.k_empty[kst], ((kt / K3_NK) & 1) ^ 1) &&
-             mbar_wait_warp(&sm.v_empty[vst], ((kt / K3_NV) & 1) ^ 1);
+        const int st = kt % NS;
+        ok = mbar_wait_warp(&empty[st], ((kt / NS) & 1) ^ 1);
         if (!ok) break;
         const int n = I.nres[s] - t0 < 128 ? I.nres[s] - t0 : 128;
-        if (leader) {
-          sm.desc[kst][0] = 1 << s;
-          sm.desc[kst][1] = 0;
-          sm.desc[kst][2] = n;
+        if (ROLE == 0 && leader) {
+          sm.desc[st][0] = 1 << s;
+          sm.desc[st][1] = 0;
+          sm.desc[st][2] = n;
         }
-        k3_gather<D>(sm, a, I.g, cols + t0, n, kst, vst);
-        if (leader) { mbar_arrive(&sm.k_full[kst]); mbar_arrive(&sm.v_full[vst]); }
+        k3_gather<D>(stage_buf(st), src, a, I.g, cols + t0, n);
+        if (leader) mbar_arrive(&full[st]);
         ++kt;
       }
     }
     // key blocks: union of both slots' lists
     int lo = 1 << 30, hi = -1;
+#pragma unroll
     for (int s = 0; s < 2; ++s)
       if (I.ntiles[s] > 0 && I.hi[s] >= I.lo[s]) { lo = min(lo, I.lo[s]); hi = max(hi, I.hi[s]); }
     for (int w = lo >> 5; w <= (hi >> 5) && hi >= 0 && ok; ++w) {
-      uint32_t m[2];
-      for (int s = 0; s < 2; ++s) {
-        m[s] = (I.ntiles[s] > 0) ? range_bits(w, I.lo[s], I.hi[s]) : 0u;
-        if (m[s] && a.mask) m[s] &= a.mask[((int64_t)I.h * a.nqb + I.qb[s]) * a.nkw + w];
+      uint32_t m0 = (I.ntiles[0] > 0) ? range_bits(w, I.lo[0], I.hi[0]) : 0u;
+      uint32_t m1 = (I.ntiles[1] > 0) ? range_bits(w, I.lo[1], I.hi[1]) : 0u;
+      if (a.mask) {
+        if (m0) m0 &= a.mask[((int64_t)I.h * a.nqb + I.qb[0]) * a.nkw + w];
+        if (m1) m1 &= a.mask[((int64_t)I.h * a.nqb + I.qb[1]) * a.nkw + w];
       }
-      uint32_t u = m[0] | m[1];
+      uint32_t u = m0 | m1;
       while (u && ok) {
         const int b = __ffs(u) - 1;
         u &= u - 1;
         const int kb = 32 * w + b;
-        const int flags = (int)((m[0] >> b) & 1u) | (int)(((m[1] >> b) & 1u) << 1);
-        const int diag = (int)(kb == I.B[0]) | ((int)(kb == I.B[1]) << 1);
-        const int kst = kt % K3_NK, vst = kt % K3_NV;
-        ok = mbar_wait_warp(&sm.k_empty[kst], ((kt / K3_NK) & 1) ^ 1);
+        const int st = kt % NS;
+        ok = mbar_wait_warp(&empty[st], ((kt / NS) & 1) ^ 1);
         if (!ok) break;
         const int y = (int)((int64_t)I.g * a.ld_tokens + (int64_t)kb * 128);
         if (leader) {
-          sm.desc[kst][0] = flags;
-          sm.desc[kst][1] = diag;
-          sm.desc[kst][2] = 128;
-          mbar_expect_tx(&sm.k_full[kst], TILE);
+          if (ROLE == 0) {
+            sm.desc[st][0] = (int)((m0 >> b) & 1u) | (int)(((m1 >> b) & 1u) << 1);
+            sm.desc[st][1] = (int)(kb == I.B[0]) | ((int)(kb == I.B[1]) << 1);
+            sm.desc[st][2] = 128;
+          }
+          mbar_expect_tx(&full[st], TILE);
 #pragma unroll
-          for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(sm.k[kst] + hf * 16384, mk, &sm.k_full[kst], 64 * hf, y);
-        }
-        ok = mbar_wait_warp(&sm.v_empty[vst], ((kt / K3_NV) & 1) ^ 1);
-        if (!ok) break;
-        if (leader) {
-          mbar_expect_tx(&sm.v_full[vst], TILE);
-#pragma unroll
-          for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(sm.v[vst] + hf * 16384, mv, &sm.v_full[vst], 64 * hf, y);
+          for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(stage_buf(st) + hf * 16384, map, &full[st], 64 * hf, y);
         }
         ++kt;
       }
@@ -247,7 +260,8 @@ __device__ void k3_producer(K3Smem<D>& sm, const K3Args& a, const CUtensorMap* m
 }
 
 // --------------------------------------------------------------------------------------
-// MMA warp (one thread issues). Per-slot state lives in registers (static slot indices).
+// MMA warp. The whole warp runs the loop (waits, bookkeeping and descriptors are warp-
+// uniform); one elected lane issues each tcgen05.mma / commit / arrive.
 // --------------------------------------------------------------------------------------
 struct K3Slot {
   int pend_v = -1;            // V stage of the slot's pending PV (-1: none)
@@ -257,63 +271,84 @@ struct K3Slot {
   uint32_t qn = 0, pn = 0, pvd_issued = 0, pvd_waited = 0;
 };
 
+struct K3Desc {
+  uint64_t q[2], k[K3_NK], v[K3_NV];   // 128B-swizzle descriptors of the tile bases
+  // stage selection by value (no dynamically indexed local arrays)
+  __device__ __forceinline__ uint64_t kd(int st) const {
+    static_assert(K3_NK == 2, "two K stages");
+    return st ? k[1] : k[0];
+  }
+  __device__ __forceinline__ uint64_t vd(int st) const {
+    static_assert(K3_NV == 2, "two V stages");
+    return st ? v[1] : v[0];
+  }
+};
+
 // PV of the slot's pending tile: O (+)= P V, P read from tensor memory.
 template <int D, int S>
-__device__ __forceinline__ bool k3_pv(K3Smem<D>& sm, K3Slot& sl, uint32_t tb, uint32_t& v_users) {
+__device__ __forceinline__ bool k3_pv(K3Smem<D>& sm, const K3Desc& dsc, K3Slot& sl, uint32_t tb,
+                                      uint32_t& v_users) {
   constexpr uint32_t IDESC_PV = idesc_f16(128, D, 1);
-  if (!mbar_wait(&sm.p_full[S], sl.pn & 1)) return false;
+  if (!mbar_wait_warp(&sm.p_full[S], sl.pn & 1)) return false;
   ++sl.pn;
   const int vst = sl.pend_v;
-  if (!mbar_wait(&sm.v_full[vst], (sl.pend_kt / K3_NV) & 1)) return false;
+  if (!mbar_wait_warp(&sm.v_full[vst], (sl.pend_kt / K3_NV) & 1)) return false;
   tc_fence_after();
   const uint32_t o_t = tb + 256u * S + 128u, p_t = tb + 256u * S;
-  const uint32_t vbase = smem_u32(sm.v[vst]);
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    mma_ts(o_t, p_t + kk * 8u, sdesc_sw128(vbase + kk * 2048u, 16384u, 1024u), IDESC_PV,
-           (sl.o_started || kk > 0) ? 1u : 0u);
-  sl.o_started = true;
-  // P lives in S's columns: the slot's next QK^T may overwrite them only after this PV read them
-  mma_commit(&sm.pv_done[S]);
-  ++sl.pvd_issued;
-  if (sl.pend_last) { mma_commit(&sm.o_done[S]); sl.o_started = false; }
+  const uint64_t vd = dsc.vd(vst);
   const uint32_t sh = 4u * (uint32_t)vst;
   const uint32_t u = ((v_users >> sh) & 0xFu) - 1u;
+  if (elect_one()) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)   // 16 keys = 16 rows of 128 B per step (2048 B, >> 4 = 128)
+      mma_ts(o_t, p_t + kk * 8u, vd + (uint64_t)(kk * 128), IDESC_PV,
+             (sl.o_started || kk > 0) ? 1u : 0u);
+    // P lives in S's columns: the slot's next QK^T may overwrite them only after this PV
+    mma_commit(&sm.pv_done[S]);
+    if (sl.pend_last) mma_commit(&sm.o_done[S]);
+    if (u == 0) mma_commit(&sm.v_empty[vst]);
+  }
+  __syncwarp();
+  sl.o_started = !sl.pend_last;
+  ++sl.pvd_issued;
   v_users = (v_users & ~(0xFu << sh)) | (u << sh);
-  if (u == 0) mma_commit(&sm.v_empty[vst]);
   sl.pend_v = -1;
   return true;
 }
 
 // S = Q K^T for the slot on K stage kst.
 template <int D, int S>
-__device__ __forceinline__ bool k3_qk(K3Smem<D>& sm, K3Slot& sl, int& rem, bool& first, int kst,
-                                      int vst, uint32_t kt, int diag, int ncols, uint32_t tb) {
+__device__ __forceinline__ bool k3_qk(K3Smem<D>& sm, const K3Desc& dsc, K3Slot& sl, int& rem,
+                                      bool& first, int kst, int vst, uint32_t kt, int diag,
+                                      int ncols, uint32_t tb) {
   constexpr uint32_t IDESC_QK = idesc_f16(128, 128, 0);
   if (first) {
-    if (!mbar_wait(&sm.q_full[S], sl.qn & 1)) return false;
+    if (!mbar_wait_warp(&sm.q_full[S], sl.qn & 1)) return false;
     ++sl.qn;
     first = false;
     tc_fence_after();
   }
-  if (sl.pvd_waited < sl.pvd_issued) {
-    if (!mbar_wait(&sm.pv_done[S], sl.pvd_waited & 1)) return false;
+  if (K3_WAIT_PV_BEFORE_QK && sl.pvd_waited < sl.pvd_issued) {
+    if (!mbar_wait_warp(&sm.pv_done[S], sl.pvd_waited & 1)) return false;
     ++sl.pvd_waited;
   }
   --rem;
   const bool last = rem == 0;
-  sm.meta[S] = ((diag >> S) & 1) | (ncols << 8) | ((int)last << 16);
-  mbar_arrive(&sm.s_full[S]);
   const uint32_t s_t = tb + 256u * S;
-  const uint32_t qbase = smem_u32(sm.q[S]), kbase = smem_u32(sm.k[kst]);
+  const uint64_t qd = dsc.q[S], kd = dsc.kd(kst);
+  if (elect_one()) {
+    sm.meta[S] = ((diag >> S) & 1) | (ncols << 8) | ((int)last << 16);
+    mbar_arrive(&sm.s_full[S]);
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
-    mma_ss(s_t, sdesc_sw128(qbase + off, 16u, 1024u), sdesc_sw128(kbase + off, 16u, 1024u),
-           IDESC_QK, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < D / 16; ++kk) {
+      // 16 fp16 of K = 32 B inside a 128 B swizzle row (>> 4 = 2); halves 16 KB apart
+      const uint64_t off = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
+      mma_ss(s_t, qd + off, kd + off, IDESC_QK, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&sm.s_full[S]);
+    if (last) mma_commit(&sm.q_empty[S]);
   }
-  mma_commit(&sm.s_full[S]);
-  if (last) mma_commit(&sm.q_empty[S]);
+  __syncwarp();
   sl.pend_v = vst;
   sl.pend_kt = kt;
   sl.pend_last = last;
@@ -323,6 +358,13 @@ __device__ __forceinline__ bool k3_qk(K3Smem<D>& sm, K3Slot& sl, int& rem, bool&
 template <int D>
 __device__ void k3_mma(K3Smem<D>& sm, const K3Args& a, int nitems) {
   const uint32_t tb = sm.tmem_base;
+  K3Desc dsc;
+  dsc.q[0] = sdesc_sw128(smem_u32(sm.q[0]), 16u, 1024u);
+  dsc.q[1] = sdesc_sw128(smem_u32(sm.q[1]), 16u, 1024u);
+#pragma unroll
+  for (int i = 0; i < K3_NK; ++i) dsc.k[i] = sdesc_sw128(smem_u32(sm.k[i]), 16u, 1024u);
+#pragma unroll
+  for (int i = 0; i < K3_NV; ++i) dsc.v[i] = sdesc_sw128(smem_u32(sm.v[i]), 16384u, 1024u);
   uint32_t kt = 0;
   K3Slot s0, s1;
   uint32_t v_users = 0;       // 4 bits per V stage: PVs still to issue on it
@@ -333,26 +375,30 @@ __device__ void k3_mma(K3Smem<D>& sm, const K3Args& a, int nitems) {
     bool first0 = true, first1 = true;
     while ((rem0 > 0 || rem1 > 0) && ok) {
       const int kst = kt % K3_NK, vst = kt % K3_NV;
-      ok = mbar_wait(&sm.k_full[kst], (kt / K3_NK) & 1);
+      // slot 0's pending PV does not need the next K tile: issue it first
+      if (s0.pend_v >= 0) ok = k3_pv<D, 0>(sm, dsc, s0, tb, v_users);
+      if (!ok) break;
+      ok = mbar_wait_warp(&sm.k_full[kst], (kt / K3_NK) & 1);
       if (!ok) break;
       tc_fence_after();
       const int flags = sm.desc[kst][0], diag = sm.desc[kst][1], ncols = sm.desc[kst][2];
       uint32_t users = 0;
-      if (ok && s0.pend_v >= 0) ok = k3_pv<D, 0>(sm, s0, tb, v_users);
-      if (ok && (flags & 1)) { ok = k3_qk<D, 0>(sm, s0, rem0, first0, kst, vst, kt, diag, ncols, tb); ++users; }
-      if (ok && s1.pend_v >= 0) ok = k3_pv<D, 1>(sm, s1, tb, v_users);
-      if (ok && (flags & 2)) { ok = k3_qk<D, 1>(sm, s1, rem1, first1, kst, vst, kt, diag, ncols, tb); ++users; }
+      if (ok && (flags & 1)) { ok = k3_qk<D, 0>(sm, dsc, s0, rem0, first0, kst, vst, kt, diag, ncols, tb); ++users; }
+      if (ok && s1.pend_v >= 0) ok = k3_pv<D, 1>(sm, dsc, s1, tb, v_users);
+      if (ok && (flags & 2)) { ok = k3_qk<D, 1>(sm, dsc, s1, rem1, first1, kst, vst, kt, diag, ncols, tb); ++users; }
       if (!ok) break;
       const uint32_t sh = 4u * (uint32_t)vst;
       v_users = (v_users & ~(0xFu << sh)) | (users << sh);
-      mma_commit(&sm.k_empty[kst]);
+      if (elect_one()) mma_commit(&sm.k_empty[kst]);
+      __syncwarp();
       ++kt;
     }
   }
-  if (ok && s0.pend_v >= 0) ok = k3_pv<D, 0>(sm, s0, tb, v_users);
-  if (ok && s1.pend_v >= 0) ok = k3_pv<D, 1>(sm, s1, tb, v_users);
-  mma_commit(&sm.drain);
-  mbar_wait(&sm.drain, 0);
+  if (ok && s0.pend_v >= 0) ok = k3_pv<D, 0>(sm, dsc, s0, tb, v_users);
+  if (ok && s1.pend_v >= 0) ok = k3_pv<D, 1>(sm, dsc, s1, tb, v_users);
+  if (elect_one()) mma_commit(&sm.drain);
+  __syncwarp();
+  mbar_wait_warp(&sm.drain, 0);
 }
 
 // --------------------------------------------------------------------------------------
@@ -395,15 +441,20 @@ __device__ void k3_softmax(K3Smem<D>& sm, const K3Args& a, int nitems) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) if (c > lim) x[c] = -INFINITY;
       }
-      // row maximum: eight independent chains of 3-input max
+      // row maximum: eight independent chains of 2-input max (the 3-input max.f32 is far
+      // slower on sm_100: measured 550 vs 115 cycles per 128-column row)
       float a8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) a8[k] = x[k];
 #pragma unroll
-      for (int c = 8; c < 128; c += 16)
+      for (int c = 8; c < 128; c += 8)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) a8[k] = fmax3(a8[k], x[c + k], x[c + 8 + k]);
-      const float mx = fmaxf(fmax3(a8[0], a8[1], a8[2]), fmax3(fmax3(a8[3], a8[4], a8[5]), a8[6], a8[7]));
+        for (int k = 0; k < 8; ++k) a8[k] = fmaxf(a8[k], x[c + k]);
+#pragma unroll
+      for (int wdt = 4; wdt >= 1; wdt /= 2)
+#pragma unroll
+        for (int k = 0; k < wdt; ++k) a8[k] = fmaxf(a8[k], a8[k + wdt]);
+      const float mx = a8[0];
       const bool need = mx > m + K3_RESCALE_THRESHOLD;
       if (__any_sync(0xFFFFFFFFu, need)) {
         const float m_new = need ? mx : m;
@@ -432,9 +483,16 @@ __device__ void k3_softmax(K3Smem<D>& sm, const K3Args& a, int nitems) {
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int j = 32 * ch + 2 * c;
-          float d0, d1;
-          f2_unpack(f2_add(f2_pack(x[j], x[j + 1]), nmu), d0, d1);
-          const float p0 = ex2(d0), p1 = ex2(d1);
+          const uint64_t dx = f2_add(f2_pack(x[j], x[j + 1]), nmu);
+          float p0, p1;
+          if ((c & 7) < K3_POLY_PAIRS_OF_8) {
+            f2_unpack(ex2_poly2(dx), p0, p1);       // FMA pipe
+          } else {
+            float d0, d1;
+            f2_unpack(dx, d0, d1);
+            p0 = ex2(d0);                           // multi-function unit
+            p1 = ex2(d1);
+          }
           acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
           pk[c] = pack_f16x2(p0, p1);
         }
@@ -504,8 +562,9 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_co
     else k3_softmax<D, 1>(sm, a, nitems);
   } else {
     regs_decrease<K3_REGS_OTHER>();
-    if (w == 8) k3_producer<D>(sm, a, &mq, &mk, &mv, nitems);
-    else if (w == 9 && lane_id() == 0) k3_mma<D>(sm, a, nitems);
+    if (w == 8) k3_producer<D, 0>(sm, a, &mq, &mk, &mv, nitems);
+    else if (w == 9) k3_mma<D>(sm, a, nitems);
+    else if (w == 10) k3_producer<D, 1>(sm, a, &mq, &mk, &mv, nitems);
   }
   tc_fence_before();
   __syncthreads();

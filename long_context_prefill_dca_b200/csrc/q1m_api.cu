@@ -699,6 +699,16 @@ q1m_status q1m_set_wait_budget(uint64_t cycles) {
 }  // extern "C"
 
 namespace {
+__global__ void selftest_exp2_kernel(const float* x, float* yp, float* ym, float* yr, int64_t n) {
+  const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 2;
+  if (i + 1 >= n + 1) return;
+  const float a = x[i], b = i + 1 < n ? x[i + 1] : 0.f;
+  float pa, pb;
+  f2_unpack(ex2_poly2(f2_pack(a, b)), pa, pb);
+  yp[i] = pa; ym[i] = ex2(a); yr[i] = exp2f(a);
+  if (i + 1 < n) { yp[i + 1] = pb; ym[i + 1] = ex2(b); yr[i + 1] = exp2f(b); }
+}
+
 // one warp waits on a barrier that no thread and no copy ever arrives on
 __global__ void selftest_wait_kernel() {
   __shared__ uint64_t bar;
@@ -707,6 +717,16 @@ __global__ void selftest_wait_kernel() {
   mbar_wait(&bar, 0);
 }
 }  // namespace
+
+extern "C" q1m_status q1m_selftest_exp2(const float* x, float* yp, float* ym, float* yr, int64_t n,
+                                        void* stream) {
+  if (!x || !yp || !ym || !yr || n <= 0) return fail(Q1M_ERR_INVALID, "bad arguments");
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  selftest_exp2_kernel<<<blocks_for((n + 1) / 2, 256), 256, 0, S(stream)>>>(x, yp, ym, yr, n);
+  Q1M_LAUNCHED();
+  return Q1M_OK;
+}
 
 extern "C" q1m_status q1m_selftest_wait_timeout(uint64_t cycles, void* stream) {
   Dev dev;

@@ -12,6 +12,7 @@
 #include <stdint.h>
 
 #include "../../include/q1m.h"
+#include "exp2_poly.h"
 
 namespace q1m {
 
@@ -30,6 +31,18 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 }
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
+
+// One lane of a converged warp is elected (the same lane every time); the rest of the warp
+// keeps executing the same code, so warp-uniform values stay in uniform registers.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 
 // ---------------------------------------------------------------------------------------
@@ -342,6 +355,36 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe instead of the multi-function unit:
+// Cody-Waite style reduction x = n + r (n = round(x) by the 1.5 * 2^23 addition trick,
+// r in [-1/2, 1/2]), 2^r by the degree-4 polynomial of exp2_poly.h (relative error
+// 3.1e-6), and 2^n applied by adding n to the exponent field. Inputs are clamped at -127 so
+// the exponent add cannot wrap (2^-127 is far below fp16 resolution; -inf gives 2^-127).
+__device__ __forceinline__ uint64_t ex2_poly2(uint64_t x2) {
+  float a, b;
+  f2_unpack(x2, a, b);
+  const uint64_t xc = f2_pack(fmaxf(a, -127.f), fmaxf(b, -127.f));
+  const uint64_t t = f2_add(xc, f2_pack(12582912.f, 12582912.f));   // n + 1.5 * 2^23
+  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));  // n, exact
+  const uint64_t r = f2_fma(n, f2_pack(-1.f, -1.f), xc);             // x - n, exact
+  uint64_t p = f2_pack(Q1M_EXP2_C4, Q1M_EXP2_C4);
+  p = f2_fma(p, r, f2_pack(Q1M_EXP2_C3, Q1M_EXP2_C3));
+  p = f2_fma(p, r, f2_pack(Q1M_EXP2_C2, Q1M_EXP2_C2));
+  p = f2_fma(p, r, f2_pack(Q1M_EXP2_C1, Q1M_EXP2_C1));
+  p = f2_fma(p, r, f2_pack(Q1M_EXP2_C0, Q1M_EXP2_C0));
+  float pa, pb, ta, tb;
+  f2_unpack(p, pa, pb);
+  f2_unpack(t, ta, tb);
+  // the low mantissa bits of t hold n: (bits(t) << 23) == n << 23 modulo 2^32
+  return f2_pack(__int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23)),
+                 __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23)));
 }
 
 // Two fp32 -> packed fp16x2 (lo in bits 0..15), round to nearest even.

@@ -71,6 +71,7 @@ SIGNATURES = {
     "q1m_profile_read": (c_int, [ctypes.POINTER(c_dbl), ctypes.POINTER(c_i64)]),
     "q1m_launch_count": (c_u64, []),
     "q1m_selftest_wait_timeout": (c_int, [c_u64, c_vp]),
+    "q1m_selftest_exp2": (c_int, [c_vp, c_vp, c_vp, c_vp, c_i64, c_vp]),
 }
 
 _LIB = None
@@ -247,6 +248,11 @@ def profile_read() -> dict:
 
 def launch_count() -> int:
     return int(library().q1m_launch_count())
+
+
+def selftest_exp2(x, y_poly, y_mufu, y_ref, stream=None) -> None:
+    _call("q1m_selftest_exp2", ptr(x), ptr(y_poly), ptr(y_mufu), ptr(y_ref), x.numel(),
+          stream_handle(stream))
 
 
 def version() -> str:

@@ -283,3 +283,22 @@ def test_bounded_wait_returns_timeout_and_library_recovers():
     torch.cuda.synchronize()
     q1m.check_status()
     assert np.abs(out.cpu().numpy() - c["out"]).max() <= MAX_ABS
+
+
+def test_fma_pipe_exp2_error_bound():
+    """The kernel's polynomial 2^x against CUDA's exp2f and fp64, over the range the
+    softmax feeds it (x - max <= 8 by the lazy rescale; very negative values underflow)."""
+    xs = np.concatenate([np.linspace(-130.0, 8.0, 1_000_003), np.arange(-127, 9, dtype=np.float64),
+                         np.arange(-127, 9) + 0.5, [-np.inf]]).astype(np.float32)
+    x = torch.from_numpy(xs).cuda()
+    yp, ym, yr = torch.empty_like(x), torch.empty_like(x), torch.empty_like(x)
+    q1m.selftest_exp2(x, yp, ym, yr)
+    torch.cuda.synchronize()
+    yp, yr = yp.cpu().numpy().astype(np.float64), yr.cpu().numpy().astype(np.float64)
+    ref = np.exp2(xs.astype(np.float64))
+    normal = xs >= -126.0
+    rel = np.abs(yp[normal] - ref[normal]) / ref[normal]
+    assert rel.max() < 4e-6, rel.max()
+    assert np.abs(yr[normal] - ref[normal]).max() / ref[normal].max() < 1e-6
+    # below -126 the result is tiny (no wrap-around), as is 2^-inf
+    assert np.all(yp[~normal] >= 0) and np.all(yp[~normal] < 1.2e-38)
