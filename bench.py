@@ -46,6 +46,22 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The slowest rank's value (all ranks call this in the same order)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the work of every rank over the slowest rank's step time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -212,6 +228,21 @@ def oracle_sample(w, x, dense_pairs_total, n_rows=4):
     return t_layer, desc, pairs_total
 
 
+def estimator_work(w) -> dict:
+    """Algorithmic work of the vertical-slash estimator over all prefill chunks: bytes (two
+    passes over the fp16 key prefix, the estimator query rows, the fp32 scores written),
+    tensor FLOPs (two passes of 2 * rows * keys * D per KV-group row set) and exponentials."""
+    D, hq, hkv = w.head_dim, w.n_q_heads, w.n_kv_heads
+    byts = flops = exps = 0.0
+    for s0 in range(0, w.seq_len, w.prefill_chunk):
+        e = min(w.seq_len, s0 + w.prefill_chunk)
+        rows = min(w.vs_last_q, e - s0)
+        byts += 2 * e * hkv * D * 2 + rows * hq * D * 2 + 2 * hq * e * 4
+        flops += 2 * 2.0 * rows * hq * e * D
+        exps += 2.0 * rows * hq * e
+    return {"bytes": byts, "flops": flops, "exps": exps}
+
+
 def dense_pairs(w) -> float:
     n = float(w.seq_len)
     return n * (n + 1) / 2 * w.n_q_heads
@@ -320,12 +351,8 @@ def main():
     q1m.profile_enable(False)
     clk = clocks.stop()
     q1m.check_status(stream)
-    ms_total = ev0.elapsed_time(ev1)
-    t = torch.tensor([ms_total], device=device, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step = float(t.item()) / args.steps
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1), world, device) / args.steps
+    value = job_tflops(flops, world, ms_step)
 
     # e2e: the same layer through the host-buffer entry point, copies included
     e2e = None
@@ -345,12 +372,9 @@ def main():
             hl(pin["q"], pin["k"], pin["v"], out_h, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize(device)
-        te = torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], device=device, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        ms_e2e = float(te.item())
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, device)
         h2d = sum(v.numel() * v.element_size() for v in pin.values())
-        e2e = {"value": flops * world / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_tflops(flops, world, ms_e2e), "unit": UNIT,
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": args.e2e_steps}
         del hl, pin, out_h
@@ -368,6 +392,18 @@ def main():
                 "layer_frac": value / world / sustained}
     stages = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
               for k, v in prof.items()}
+    estimator = None
+    if not w.dense and prof["estimate"][0] > 0:
+        ew = estimator_work(w)
+        t_est = prof["estimate"][0] / args.steps * 1e-3
+        estimator = {"ms_per_step": t_est * 1e3,
+                     "algorithmic_bytes": ew["bytes"], "gbs": ew["bytes"] / t_est / 1e9,
+                     "frac_hbm": ew["bytes"] / t_est / 1e9 / hbm,
+                     "tflops": ew["flops"] / t_est / 1e12,
+                     "frac_tensor": ew["flops"] / t_est / 1e12 / sustained,
+                     "gexp_per_s": ew["exps"] / t_est / 1e9,
+                     "note": "two tcgen05 passes over the key prefix; at D=128 with 7 Q heads "
+                             "per KV head the tensor and exponential work, not HBM, bound it"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -390,7 +426,8 @@ def main():
                        "l2": "inputs (9.6 GB) far larger than L2 (126 MB); no flush",
                        "attended_pairs": pairs, "block_density": density,
                        "ms_per_layer": ms_step},
-            "roofline": roofline, "stages": stages, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "estimator": estimator, "stages": stages,
+            "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches), "clocks": clk}
     if rank == 0:
         print(json.dumps(line), flush=True)

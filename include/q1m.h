@@ -227,6 +227,15 @@ q1m_status q1m_lse_merge(const float* o_part, const float* lse_part, int n_parts
                          int n_q_heads, int head_dim, int out_dtype, const q1m_params* p,
                          void* out, float* lse, void* stream);
 
+/* Attention recall of the sparse selection ([P2] 四 稀疏注意力机制: sparsity refinement keeps
+ * the accuracy loss of the sparse configuration small): for every row, the share of the
+ * dense softmax mass that the attended set A(i) keeps,
+ *   recall_i = sum_{j in A(i)} softmax_j(l(i, .)) = exp(lse_sparse_i - lse_dense_i),
+ * from the natural-log lse outputs of a sparse and a dense run of the same layer (n values,
+ * device fp32). recall: device fp32 [n], in [0, 1]. */
+q1m_status q1m_attention_recall(const float* lse_sparse, const float* lse_dense, int64_t n,
+                                float* recall, void* stream);
+
 /* ---------------------------------------------------------------------------------------
  * Status
  * ------------------------------------------------------------------------------------- */

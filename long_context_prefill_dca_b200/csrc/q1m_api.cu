@@ -699,6 +699,14 @@ q1m_status q1m_set_wait_budget(uint64_t cycles) {
 }  // extern "C"
 
 namespace {
+__global__ void recall_kernel(const float* __restrict__ ls, const float* __restrict__ ld, int64_t n,
+                              float* __restrict__ r) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float d = ls[i] - ld[i];
+  r[i] = d >= 0.f ? 1.f : expf(d);
+}
+
 __global__ void selftest_exp2_kernel(const float* x, float* yp, float* ym, float* yr, int64_t n) {
   const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 2;
   if (i + 1 >= n + 1) return;
@@ -717,6 +725,16 @@ __global__ void selftest_wait_kernel() {
   mbar_wait(&bar, 0);
 }
 }  // namespace
+
+extern "C" q1m_status q1m_attention_recall(const float* ls, const float* ld, int64_t n, float* r,
+                                           void* stream) {
+  if (!ls || !ld || !r || n <= 0) return fail(Q1M_ERR_INVALID, "bad arguments");
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  recall_kernel<<<blocks_for(n, 256), 256, 0, S(stream)>>>(ls, ld, n, r);
+  Q1M_LAUNCHED();
+  return Q1M_OK;
+}
 
 extern "C" q1m_status q1m_selftest_exp2(const float* x, float* yp, float* ym, float* yr, int64_t n,
                                         void* stream) {

@@ -63,6 +63,7 @@ SIGNATURES = {
                                               c_vp]),
     "q1m_lse_merge": (c_int, [c_vp, c_vp, c_int, c_i64, c_i64, c_i64, c_i64, c_int, c_int, c_int,
                               PP, c_vp, c_vp, c_vp]),
+    "q1m_attention_recall": (c_int, [c_vp, c_vp, c_i64, c_vp, c_vp]),
     "q1m_status_poll": (c_int, [c_vp]),
     "q1m_last_error": (ctypes.c_char_p, []),
     "q1m_version": (ctypes.c_char_p, []),
@@ -210,6 +211,11 @@ def lse_merge(o_part, lse_part, n_parts, ld_rows, s0, e, n, hq, d, out_dtype, p,
               stream=None):
     _call("q1m_lse_merge", ptr(o_part), ptr(lse_part), n_parts, ld_rows, s0, e, n, hq, d,
           out_dtype, ctypes.byref(p) if p is not None else None, ptr(out), ptr(lse),
+          stream_handle(stream))
+
+
+def attention_recall(lse_sparse, lse_dense, recall, stream=None) -> None:
+    _call("q1m_attention_recall", ptr(lse_sparse), ptr(lse_dense), lse_sparse.numel(), ptr(recall),
           stream_handle(stream))
 
 

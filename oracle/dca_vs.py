@@ -323,6 +323,20 @@ class Oracle:
         p, lse = softmax_rows(l)
         return p @ self.v[: imax + 1, h // self.cfg.group, :], lse
 
+    def recall_rows(self, rows: np.ndarray, h: int, sel: ChunkSelection) -> np.ndarray:
+        """Share of the dense softmax mass of each row that its attended set A(i) keeps
+        ([P2] 四 稀疏注意力机制: sparsity refinement limits the accuracy loss)."""
+        rows = np.asarray(rows)
+        imax = int(rows.max())
+        js = np.arange(imax + 1)
+        l = dca_logits(self.q_rows(rows, h), rows, self.krot(h // self.cfg.group)[: imax + 1],
+                       js, self.cfg)
+        res = np.zeros(len(rows))
+        for r, i in enumerate(rows):
+            p, _ = softmax_rows(l[[r], : i + 1])
+            res[r] = float(np.sum(p[0][self.attended(int(i), h, sel)]))
+        return res
+
     # -- whole layer -----------------------------------------------------------------------
     def run(self, rows_by_head=None, batch: int = 32):
         """Run the layer. rows_by_head: None (every row of every head) or a dict

@@ -383,3 +383,23 @@ def check_attended_set() -> bool:
         for j in range(i + 1):
             ok &= bool(m[j]) == (crossed[j // bs] or j in vset)
     return bool(ok)
+
+
+def check_recall() -> float:
+    """Recall is 1 for a full budget and equals exp(lse_sparse - lse_dense) otherwise."""
+    cfg = tiny(seq_len=260, dca_chunk=80, local_window=16, vs_vertical=4, vs_slash=12,
+               vs_force_local=4, prefill_chunk=260)
+    q, k, v = rand_qkv(cfg, 16)
+    orc = O.Oracle(q, k, v, cfg)
+    sel = orc.select_chunk(0, cfg.seq_len)
+    rows = np.array([3, 70, 129, 200, 259])
+    rec = orc.recall_rows(rows, 1, sel)
+    _, lse_s = orc.attend_rows(rows, 1, sel)
+    dense = O.Oracle(q, k, v, cfg.with_(vs_vertical=0, vs_slash=0))
+    _, lse_d = dense.attend_rows(rows, 1, O.ChunkSelection(0, cfg.seq_len))
+    full = cfg.with_(vs_vertical=10**6, vs_slash=10**6)
+    of = O.Oracle(q, k, v, full)
+    sf = of.select_chunk(0, cfg.seq_len)
+    return max(float(np.max(np.abs(rec - np.exp(lse_s - lse_d)))),
+               float(np.max(np.abs(of.recall_rows(rows, 1, sf) - 1.0))),
+               float(max(0.0, np.max(rec) - 1.0)))

@@ -1,0 +1,103 @@
+"""Edge cases of the CUDA path against the fp64 oracle: sequences shorter than one tile,
+one prefill chunk or 128-row chunks, a zero local window, one Q head per KV head, budgets at
+or above the candidate count, a slash-only budget, few estimator rows, s < 1, ragged tails;
+the host-buffer entry point; the device-side range check."""
+import numpy as np
+import pytest
+import torch
+
+from long_context_prefill_dca_b200 import q1m
+from long_context_prefill_dca_b200.layer import HostLayer, Layer
+from oracle import dca_vs as O
+from synth import configs as C
+from synth import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, MEAN_REL = 2e-2, 1e-3
+
+BASE = C.Workload(name="edge", seq_len=700, n_q_heads=4, n_kv_heads=2, head_dim=128,
+                  in_dtype="bf16", rope_base=1e4, dca_chunk=384, local_window=128, yarn_s=2.0,
+                  prefill_chunk=256, vs_vertical=20, vs_slash=70, sinks=4, bands=2,
+                  band_hi=300, seed=0x5EED0100)
+
+EDGES = [
+    BASE.with_(name="seq1-dense", seq_len=1, vs_vertical=0, vs_slash=0, sinks=0, bands=0),
+    BASE.with_(name="seq5-sparse", seq_len=5, sinks=0, bands=0),
+    BASE.with_(name="seq100-sparse", seq_len=100, sinks=2, bands=0),
+    BASE.with_(name="seq128-exact", seq_len=128, bands=0),
+    BASE.with_(name="one-chunk", prefill_chunk=1024),
+    BASE.with_(name="chunk128", prefill_chunk=128),
+    BASE.with_(name="window0", local_window=0, dca_chunk=256),
+    BASE.with_(name="mha-d64", n_q_heads=3, n_kv_heads=3, head_dim=64, in_dtype="f32"),
+    BASE.with_(name="gqa7", n_q_heads=7, n_kv_heads=1, seq_len=520),
+    BASE.with_(name="full-budget", vs_vertical=10**6, vs_slash=10**6),
+    BASE.with_(name="slash-only", vs_vertical=0, vs_slash=40),
+    BASE.with_(name="last-q-16", vs_last_q=16, vs_force_local=8),
+    BASE.with_(name="no-yarn", yarn_s=0.5),
+    BASE.with_(name="ragged-many", seq_len=1111, prefill_chunk=384),
+]
+
+
+def oracle_out(w, x):
+    orc = O.Oracle(x["q"], x["k"], x["v"], w)
+    out, lse, _ = orc.run()
+    return (np.stack([out[h] for h in range(w.n_q_heads)], axis=1),
+            np.stack([lse[h] for h in range(w.n_q_heads)], axis=0))
+
+
+def rel(a, b):
+    return float(np.sum(np.abs(a - b)) / max(np.sum(np.abs(b)), 1e-30))
+
+
+@pytest.mark.parametrize("w", EDGES, ids=lambda w: w.name)
+def test_edge_case_matches_oracle(w):
+    x = I.generate(w)
+    g = {k: t.cuda() for k, t in x.items()}
+    lse = torch.empty(w.n_q_heads, w.seq_len, device="cuda")
+    out = Layer(w)(g["q"], g["k"], g["v"], lse=lse)
+    torch.cuda.synchronize()
+    q1m.check_status()
+    ref, ref_lse = oracle_out(w, x)
+    got = out.cpu().numpy()
+    assert np.all(np.isfinite(got))
+    err = np.abs(got - ref)
+    print(f"{w.name}: max-abs {err.max():.2e} mean-rel {rel(got, ref):.2e}")
+    assert err.max() <= MAX_ABS and rel(got, ref) <= MEAN_REL
+    assert np.abs(lse.cpu().numpy() - ref_lse).max() <= 2e-3
+
+
+def test_host_buffer_entry_point_matches_device_entry_point():
+    w = BASE
+    x = I.generate(w)
+    g = {k: t.cuda() for k, t in x.items()}
+    dev = Layer(w)(g["q"], g["k"], g["v"]).cpu()
+    pin = {k: v.pin_memory() for k, v in x.items()}
+    out_h = torch.empty(dev.shape, dtype=dev.dtype).pin_memory()
+    lse_h = torch.empty(w.n_q_heads, w.seq_len).pin_memory()
+    HostLayer(w)(pin["q"], pin["k"], pin["v"], out_h, lse_h)
+    assert torch.equal(out_h, dev)
+    assert torch.isfinite(lse_h).all()
+
+
+def test_fp16_range_overflow_is_reported():
+    """Keys far beyond fp16 range latch Q1M_ERR_RANGE in the rotation stage."""
+    w = BASE.with_(vs_vertical=0, vs_slash=0)
+    x = I.generate(w)
+    x["k"][3, 0, 5] = 1e30 if w.in_dtype == "f32" else torch.tensor(3e38).to(torch.bfloat16)
+    g = {k: t.cuda() for k, t in x.items()}
+    Layer(w)(g["q"], g["k"], g["v"])
+    assert q1m.status_poll() == -6
+    assert q1m.status_poll() == 0          # the latch clears on read
+
+
+def test_nan_score_is_reported():
+    w = BASE
+    vert = torch.rand(w.n_q_heads, 300, device="cuda")
+    slash = torch.rand(w.n_q_heads, 300, device="cuda")
+    vert[1, 17] = float("nan")
+    V = torch.empty(w.n_q_heads, w.vs_vertical, dtype=torch.int32, device="cuda")
+    S = torch.empty(w.n_q_heads, w.vs_slash, dtype=torch.int32, device="cuda")
+    q1m.vs_select(vert, slash, 300, 300, w.n_q_heads, q1m.params(w), V, S)
+    assert q1m.status_poll() == -6
+    assert q1m.status_poll() == 0

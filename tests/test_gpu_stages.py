@@ -302,3 +302,27 @@ def test_fma_pipe_exp2_error_bound():
     assert np.abs(yr[normal] - ref[normal]).max() / ref[normal].max() < 1e-6
     # below -126 the result is tiny (no wrap-around), as is 2^-inf
     assert np.all(yp[~normal] >= 0) and np.all(yp[~normal] < 1.2e-38)
+
+
+@pytest.mark.parametrize("w", SPARSE, ids=lambda w: w.name)
+def test_attention_recall_matches_oracle(w):
+    """recall_i = exp(lse_sparse - lse_dense) from the GPU against the oracle's share of the
+    dense softmax mass kept by A(i), on the oracle's selection."""
+    c = case(w)
+    _, lse_s = run_oracle_fed(w, c)
+    wd = w.with_(vs_vertical=0, vs_slash=0)
+    lse_d = torch.empty(w.n_q_heads, w.seq_len, device="cuda")
+    Layer(wd)(c["g"]["q"], c["g"]["k"], c["g"]["v"], lse=lse_d)
+    r = torch.empty_like(lse_d)
+    q1m.attention_recall(torch.from_numpy(lse_s).cuda(), lse_d, r)
+    torch.cuda.synchronize()
+    q1m.check_status()
+    r = r.cpu().numpy()
+    g = np.random.default_rng(3)
+    orc = c["orc"]
+    for sel in c["sels"]:
+        for h in range(w.n_q_heads):
+            rows = np.sort(g.choice(np.arange(sel.s0, sel.e), size=16, replace=False))
+            ref = orc.recall_rows(rows, h, sel)
+            assert np.abs(r[h, rows] - ref).max() < 5e-3, (sel.s0, h)
+    assert np.all((r > 0) & (r <= 1.0))

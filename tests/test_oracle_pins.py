@@ -72,3 +72,7 @@ def test_block_mask_brute_force():
 
 def test_attended_set_enumeration():
     assert C.check_attended_set()
+
+
+def test_recall_identity_and_full_budget():
+    assert C.check_recall() < 1e-12
