@@ -33,6 +33,29 @@ METRIC = "DCA+sparse prefill attn ms/layer & effective TFLOP/s at 1M tok; % BF16
 UNIT = "TFLOP/s"
 
 
+KERNEL_SOURCES = ("attn_tc.cuh", "q1m_device.cuh", "exp2_poly.h")
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "block_sparse_attn_dram_7b-1m.md")
+
+
+def kernel_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary of the 7B@1M layer, or
+    None when the workload differs or the kernel's sources changed since the capture (their
+    sha256 is recorded beside the figure)."""
+    import hashlib
+    if workload != "7b-1m" or not os.path.exists(TRAFFIC_PROFILE):
+        return None
+    rec = {}
+    for line in open(TRAFFIC_PROFILE):
+        if ":" in line and line.split(":", 1)[0] in ("traffic_per_launch_bytes", "kernel_source_sha256"):
+            k, v = line.split(":", 1)
+            rec[k] = v.strip()
+    csrc = os.path.join(ROOT, "long_context_prefill_dca_b200", "csrc")
+    h = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read() for f in KERNEL_SOURCES)).hexdigest()
+    if rec.get("kernel_source_sha256") != h or "traffic_per_launch_bytes" not in rec:
+        return None
+    return float(rec["traffic_per_launch_bytes"])
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -386,7 +409,8 @@ def main():
     achieved = (flops * args.steps / attn_n) / (attn_ms / attn_n * 1e-3) / 1e12 if attn_n else None
     roofline = {"bound": "tensor", "kernel": "block_sparse_attn_kernel<128>",
                 "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
-                "frac": achieved / sustained if achieved else None, "traffic": None,
+                "frac": achieved / sustained if achieved else None, "traffic": kernel_traffic(w.name),
+                "traffic_unit": "DRAM bytes per launch (ncu, profiles/block_sparse_attn_dram_7b-1m.md)",
                 "peak_source": f"{src} bf16 sustained (MEASURED_PEAKS.json); fp16 operands run at the bf16 rate",
                 "frac_of_burst": achieved / burst if achieved else None,
                 "layer_frac": value / world / sustained}

@@ -76,3 +76,21 @@ def test_reference_arm_line_on_rank0():
     assert line["impl"] == "reference" and line["value"] > 0 and line["higher_is_better"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+
+
+def test_kernel_traffic_tracks_the_capture(tmp_path, monkeypatch):
+    """The roofline traffic figure comes from the committed ncu summary only while the
+    kernel's sources hash to the value recorded beside it, and only for its workload."""
+    import bench
+    assert bench.kernel_traffic("7b-128k") is None
+    fake = tmp_path / "p.md"
+    fake.write_text("traffic_per_launch_bytes: 123\nkernel_source_sha256: 00\n")
+    monkeypatch.setattr(bench, "TRAFFIC_PROFILE", str(fake))
+    assert bench.kernel_traffic("7b-1m") is None
+    import hashlib
+    import os
+    csrc = os.path.join(bench.ROOT, "long_context_prefill_dca_b200", "csrc")
+    h = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read()
+                                for f in bench.KERNEL_SOURCES)).hexdigest()
+    fake.write_text(f"traffic_per_launch_bytes: 123\nkernel_source_sha256: {h}\n")
+    assert bench.kernel_traffic("7b-1m") == 123.0
