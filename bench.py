@@ -66,6 +66,9 @@ def parse():
     ap.add_argument("--out-dtype", default="bf16", choices=["bf16", "f32"])
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--equal-cost-chunks", type=int, default=0,
+                    help="K > 0: K prefill chunks of equal dense attention cost instead of the "
+                         "workload's fixed prefill chunk")
     return ap.parse_args()
 
 
@@ -98,41 +101,9 @@ def peaks():
 # attended pairs (the work the metric counts), from the layer's own block masks
 # ---------------------------------------------------------------------------------------
 def attended_pairs(w, g, device):
-    """(total pairs over all rows and heads, computed-block density, per-chunk pairs).
-    Runs the same estimator / selection / mask kernels as the layer (not timed)."""
-    import numpy as np
-    import torch
-    from long_context_prefill_dca_b200.layer import Stages
-    if w.dense:
-        per = []
-        for s0 in range(0, w.seq_len, w.prefill_chunk):
-            e = min(w.seq_len, s0 + w.prefill_chunk)
-            i = np.arange(s0, e, dtype=np.float64)
-            per.append(float(np.sum(i + 1)) * w.n_q_heads)
-        return sum(per), 1.0, per
-    st = Stages(w, device=device)
-    total, blocks, causal, per = 0.0, 0.0, 0.0, []
-    for s0 in range(0, w.seq_len, w.prefill_chunk):
-        e = min(w.seq_len, s0 + w.prefill_chunk)
-        st.keys(g["k"], g["v"], s0, e)
-        vert, slash = st.estimate(g["q"], s0, e)
-        V, S = st.select(vert, slash, e)
-        _, _, cnt = st.masks(V, S, s0, e)
-        c = cnt.cpu().numpy().astype(np.float64)          # [hq, nqb, 8]
-        nqb = c.shape[1]
-        r0 = s0 + 128 * np.arange(nqb)
-        rows = np.minimum(128, e - r0).astype(np.float64)
-        nblk = c[:, :, 0] + c[:, :, 1] + c[:, :, 2]
-        nres = c[:, :, 6]
-        pairs = rows[None] * (128.0 * (nblk - 1.0) + nres) + rows[None] * (rows[None] + 1) / 2
-        per.append(float(pairs.sum()))
-        total += per[-1]
-        blocks += float(nblk.sum())
-        causal += float(((r0 // 128) + 1).sum()) * w.n_q_heads
-        del vert, slash, V, S, cnt
-    del st
-    torch.cuda.empty_cache()
-    return total, blocks / causal, per
+    """(total pairs, computed-block density, per-chunk pairs) from the layer's own masks."""
+    from long_context_prefill_dca_b200.accounting import attended_pairs as count
+    return count(w, g, device)
 
 
 # ---------------------------------------------------------------------------------------
@@ -255,10 +226,10 @@ def estimator_work(w) -> dict:
     """Algorithmic work of the vertical-slash estimator over all prefill chunks: bytes (two
     passes over the fp16 key prefix, the estimator query rows, the fp32 scores written),
     tensor FLOPs (two passes of 2 * rows * keys * D per KV-group row set) and exponentials."""
+    from long_context_prefill_dca_b200 import q1m
     D, hq, hkv = w.head_dim, w.n_q_heads, w.n_kv_heads
     byts = flops = exps = 0.0
-    for s0 in range(0, w.seq_len, w.prefill_chunk):
-        e = min(w.seq_len, s0 + w.prefill_chunk)
+    for s0, e in q1m.prefill_bounds(w):
         rows = min(w.vs_last_q, e - s0)
         byts += 2 * e * hkv * D * 2 + rows * hq * D * 2 + 2 * hq * e * 4
         flops += 2 * 2.0 * rows * hq * e * D
@@ -275,7 +246,7 @@ def run_reference(args):
     """The reference arm: the oracle as it stands on the host cores, bounded samples."""
     from synth import configs as C
     from synth import inputs as I
-    w = C.BY_NAME[args.workload]
+    w = C.BY_NAME[args.workload].with_(equal_cost_chunks=args.equal_cost_chunks)
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -327,7 +298,8 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=600),
                                 device_id=device)
-    w = C.BY_NAME[args.workload].with_(out_dtype=args.out_dtype)
+    w = C.BY_NAME[args.workload].with_(out_dtype=args.out_dtype,
+                                        equal_cost_chunks=args.equal_cost_chunks)
     q1m.library()
 
     x = I.generate(w)
@@ -444,6 +416,9 @@ def main():
                        "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
                        "dca_chunk": w.dca_chunk, "local_window": w.local_window,
                        "yarn_s": w.yarn_s, "prefill_chunk": w.prefill_chunk,
+                       "chunking": (f"equal-cost x{w.equal_cost_chunks}" if w.equal_cost_chunks
+                                    else "fixed"),
+                       "prefill_chunks": [list(b) for b in q1m.prefill_bounds(w)],
                        "vs_budget": [w.vs_vertical, w.vs_slash], "inputs": "bf16",
                        "mma": "f16 x f16 -> f32", "out": args.out_dtype,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",

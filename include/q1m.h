@@ -66,7 +66,24 @@ typedef struct {
   int32_t vs_last_q;       /* estimator rows: the last vs_last_q rows of a chunk (1..64)   */
   int32_t vs_force_local;  /* diagonals 0 .. vs_force_local-1 always kept (>= 1 if sparse) */
   int64_t prefill_chunk;   /* query rows per chunked-prefill step (multiple of 128)        */
+  int32_t equal_cost_chunks; /* 0: fixed chunks of prefill_chunk rows. K > 0: K chunks of
+                              * equal dense attention cost instead (q1m_prefill_bounds);
+                              * prefill_chunk is then unused                               */
 } q1m_params;
+
+/* Chunked-prefill boundaries of the layer (host function; no GPU needed). Writes the
+ * exclusive end row of each prefill chunk to ends[0 .. m-1] (chunk i covers rows
+ * [ends[i-1], ends[i]), ends[-1] = 0, ends[m-1] = seq_len) and returns m, or a negative
+ * q1m_status (Q1M_ERR_INVALID for bad arguments, Q1M_ERR_WORKSPACE when m > max_chunks).
+ *  - equal_cost_chunks == 0: chunks of prefill_chunk rows, the last one ragged.
+ *  - equal_cost_chunks == K > 0: the pages size chunks by the attention kernel's cost so
+ *    that every chunk takes about the same time ([P2] 四, pipeline-parallel optimisation,
+ *    DCPP, Figure 9); here the same sizing on one GPU. With nb = ceil(seq_len / 128) query
+ *    blocks, block b costs b + 1 key blocks (dense causal), the first m blocks cost
+ *    C(m) = m (m + 1) / 2 and T = C(nb). Chunk k (1 <= k < K) ends at block
+ *    m_k = min{ m : K C(m) >= k T } (exact integers), the last at nb; a chunk left empty
+ *    (m_k = m_{k-1}) is dropped, so m <= K. Row boundaries are 128 m_k, the last seq_len. */
+int64_t q1m_prefill_bounds(int64_t seq_len, const q1m_params* p, int64_t* ends, int64_t max_chunks);
 
 /* ---------------------------------------------------------------------------------------
  * Whole layer

@@ -160,7 +160,9 @@ q1m_status check_shape(int64_t n, int hq, int hkv, int d, const q1m_params* p) {
   if (p->local_window < 0 || p->dca_chunk <= p->local_window) return fail(Q1M_ERR_INVALID, "need 0 <= local_window < dca_chunk");
   if ((p->dca_chunk - p->local_window) % 128 != 0) return fail(Q1M_ERR_UNSUPPORTED, "dca_chunk - local_window must be a multiple of 128");
   if (p->dca_chunk > (int64_t)1 << 30) return fail(Q1M_ERR_UNSUPPORTED, "dca_chunk too large");
-  if (p->prefill_chunk <= 0 || p->prefill_chunk % 128 != 0) return fail(Q1M_ERR_INVALID, "prefill_chunk must be a positive multiple of 128");
+  if (p->equal_cost_chunks < 0) return fail(Q1M_ERR_INVALID, "equal_cost_chunks must be >= 0");
+  if (p->equal_cost_chunks == 0 && (p->prefill_chunk <= 0 || p->prefill_chunk % 128 != 0))
+    return fail(Q1M_ERR_INVALID, "prefill_chunk must be a positive multiple of 128");
   if (n > ((int64_t)1 << 31) / 8) return fail(Q1M_ERR_UNSUPPORTED, "seq_len too large");
   if ((int64_t)hkv * round_up(n, 128) >= ((int64_t)1 << 31)) return fail(Q1M_ERR_UNSUPPORTED, "n_kv_heads * seq_len too large");
   if (sparse(p)) {
@@ -171,6 +173,33 @@ q1m_status check_shape(int64_t n, int hq, int hkv, int d, const q1m_params* p) {
     if ((round_up(n, 128) / 128 + 31) / 32 > MB_MAX_NKW) return fail(Q1M_ERR_UNSUPPORTED, "seq_len too large for the block mask");
   }
   return Q1M_OK;
+}
+
+// Exclusive end rows of the prefill chunks (see q1m_prefill_bounds in the header).
+std::vector<int64_t> chunk_ends(int64_t n, const q1m_params* p) {
+  std::vector<int64_t> ends;
+  if (p->equal_cost_chunks == 0) {
+    for (int64_t s0 = 0; s0 < n; s0 += p->prefill_chunk)
+      ends.push_back(s0 + p->prefill_chunk < n ? s0 + p->prefill_chunk : n);
+    return ends;
+  }
+  using u128 = unsigned __int128;
+  const int64_t nb = (n + 127) / 128, K = p->equal_cost_chunks;
+  auto C = [](int64_t m) { return (u128)m * (u128)(m + 1) / 2; };
+  const u128 T = C(nb);
+  int64_t m = 0, prev = 0;
+  for (int64_t k = 1; k < K; ++k) {
+    while (m < nb && (u128)K * C(m) < (u128)k * T) ++m;   // smallest m with K C(m) >= k T
+    if (m > prev) { ends.push_back(128 * m < n ? 128 * m : n); prev = m; }
+  }
+  if (prev < nb) ends.push_back(n);
+  return ends;
+}
+
+int64_t max_chunk_rows(int64_t n, const q1m_params* p) {
+  int64_t s0 = 0, mx = 0;
+  for (int64_t e : chunk_ends(n, p)) { mx = e - s0 > mx ? e - s0 : mx; s0 = e; }
+  return mx;
 }
 
 float view_scale(const q1m_params* p, int d) {
@@ -214,8 +243,7 @@ struct Layout {
 Layout layout(int64_t n, int hq, int hkv, int d, const q1m_params* p) {
   Layout L{};
   L.ld_tokens = round_up(n, 128);
-  const int64_t P = p->prefill_chunk < n ? p->prefill_chunk : n;
-  L.ld_rows = round_up(P, 128);
+  L.ld_rows = round_up(max_chunk_rows(n, p), 128);
   L.nqb_max = L.ld_rows / 128;
   L.nkw_max = (L.ld_tokens / 128 + 31) / 32;
   L.nv = (int)(p->vs_vertical < n ? p->vs_vertical : n);
@@ -589,8 +617,8 @@ q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, v
       Q1M_CUDA(cudaMemsetAsync(v16 + ((int64_t)g * L.ld_tokens + n) * d, 0, (size_t)(L.ld_tokens - n) * d * 2, st));
     }
   }
-  for (int64_t s0 = 0; s0 < n; s0 += p->prefill_chunk) {
-    const int64_t e = s0 + p->prefill_chunk < n ? s0 + p->prefill_chunk : n;
+  int64_t s0 = 0;
+  for (const int64_t e : chunk_ends(n, p)) {
     pr = prof_begin(Q1M_STAGE_KEYS, st);
     Q1M_TRY(run_rope_keys(k, v, s0, e, hkv, d, p, table, k_rot, v16, L.ld_tokens, st));
     prof_end(pr, st);
@@ -623,6 +651,7 @@ q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, v
     pr = prof_begin(Q1M_STAGE_MERGE, st);
     Q1M_TRY(run_merge(o_part, lse_part, 3, L.ld_rows, s0, e, n, hq, d, p->out_dtype, Ld, out, lse, st));
     prof_end(pr, st);
+    s0 = e;
   }
   return Q1M_OK;
 }
@@ -651,6 +680,17 @@ q1m_status q1m_dca_sparse_prefill_host(const void* q_h, const void* k_h, const v
   Q1M_CUDA(cudaMemcpyAsync(out_h, dout, bo, cudaMemcpyDeviceToHost, st));
   if (lse_h) Q1M_CUDA(cudaMemcpyAsync(lse_h, dlse, (size_t)n * hq * 4, cudaMemcpyDeviceToHost, st));
   return q1m_status_poll(stream);
+}
+
+int64_t q1m_prefill_bounds(int64_t n, const q1m_params* p, int64_t* ends, int64_t max_chunks) {
+  if (!p || !ends || n <= 0 || max_chunks <= 0) return fail(Q1M_ERR_INVALID, "bad arguments");
+  if (p->equal_cost_chunks < 0) return fail(Q1M_ERR_INVALID, "equal_cost_chunks must be >= 0");
+  if (p->equal_cost_chunks == 0 && (p->prefill_chunk <= 0 || p->prefill_chunk % 128 != 0))
+    return fail(Q1M_ERR_INVALID, "prefill_chunk must be a positive multiple of 128");
+  const std::vector<int64_t> e = chunk_ends(n, p);
+  if ((int64_t)e.size() > max_chunks) return fail(Q1M_ERR_WORKSPACE, "%zu chunks > max_chunks", e.size());
+  for (size_t i = 0; i < e.size(); ++i) ends[i] = e[i];
+  return (int64_t)e.size();
 }
 
 q1m_status q1m_status_poll(void* stream) {

@@ -59,7 +59,7 @@ class Stages:
         self.p = q1m.params(w, out_dtype)
         n, hq, hkv, d = w.seq_len, w.n_q_heads, w.n_kv_heads, w.head_dim
         self.ld_tokens = _r128(n)
-        self.ld_rows = _r128(min(w.prefill_chunk, n))
+        self.ld_rows = _r128(max(e - s0 for s0, e in q1m.prefill_bounds(w)))
         self.table = torch.empty(w.dca_chunk * d, dtype=torch.float32, device=device)
         self.k_rot = torch.zeros(hkv, self.ld_tokens, d, dtype=torch.int16, device=device)
         self.v16 = torch.zeros(hkv, self.ld_tokens, d, dtype=torch.int16, device=device)

@@ -24,7 +24,8 @@ class Params(ctypes.Structure):
     _fields_ = [("in_dtype", c_i32), ("out_dtype", c_i32), ("rope_base", c_dbl),
                 ("yarn_s", c_dbl), ("dca_chunk", c_i64), ("local_window", c_i64),
                 ("vs_vertical", c_i32), ("vs_slash", c_i32), ("vs_last_q", c_i32),
-                ("vs_force_local", c_i32), ("prefill_chunk", c_i64)]
+                ("vs_force_local", c_i32), ("prefill_chunk", c_i64),
+                ("equal_cost_chunks", c_i32)]
 
 
 class Q1MError(RuntimeError):
@@ -64,6 +65,7 @@ SIGNATURES = {
     "q1m_lse_merge": (c_int, [c_vp, c_vp, c_int, c_i64, c_i64, c_i64, c_i64, c_int, c_int, c_int,
                               PP, c_vp, c_vp, c_vp]),
     "q1m_attention_recall": (c_int, [c_vp, c_vp, c_i64, c_vp, c_vp]),
+    "q1m_prefill_bounds": (c_i64, [c_i64, PP, c_vp, c_i64]),
     "q1m_status_poll": (c_int, [c_vp]),
     "q1m_last_error": (ctypes.c_char_p, []),
     "q1m_version": (ctypes.c_char_p, []),
@@ -105,7 +107,7 @@ def params(w, out_dtype: str | None = None) -> Params:
     return Params(BF16 if w.in_dtype == "bf16" else F32, BF16 if od == "bf16" else F32,
                   float(w.rope_base), float(w.yarn_s), int(w.dca_chunk), int(w.local_window),
                   int(w.vs_vertical), int(w.vs_slash), int(w.vs_last_q), int(w.vs_force_local),
-                  int(w.prefill_chunk))
+                  int(w.prefill_chunk), int(getattr(w, "equal_cost_chunks", 0)))
 
 
 def ptr(t) -> int | None:
@@ -217,6 +219,23 @@ def lse_merge(o_part, lse_part, n_parts, ld_rows, s0, e, n, hq, d, out_dtype, p,
 def attention_recall(lse_sparse, lse_dense, recall, stream=None) -> None:
     _call("q1m_attention_recall", ptr(lse_sparse), ptr(lse_dense), lse_sparse.numel(), ptr(recall),
           stream_handle(stream))
+
+
+def prefill_bounds(w) -> list[tuple[int, int]]:
+    """(s0, e) of every prefill chunk of workload w, as the library's driver loop runs them
+    (host computation; no GPU needed)."""
+    n = int(w.seq_len)
+    cap = n // 128 + 2
+    ends = (c_i64 * cap)()
+    p = params(w)
+    m = library().q1m_prefill_bounds(n, ctypes.byref(p), ends, cap)
+    if m < 0:
+        raise Q1MError("q1m_prefill_bounds", int(m), library().q1m_last_error().decode())
+    out, s0 = [], 0
+    for e in ends[:m]:
+        out.append((s0, int(e)))
+        s0 = int(e)
+    return out
 
 
 def status_poll(stream=None) -> int:

@@ -40,8 +40,7 @@ def recall(w, g) -> torch.Tensor:
 
 def summarize(w, r: torch.Tensor) -> dict:
     out = {"workload": w.name, "budget": [w.vs_vertical, w.vs_slash], "per_chunk": []}
-    for s0 in range(0, w.seq_len, w.prefill_chunk):
-        e = min(w.seq_len, s0 + w.prefill_chunk)
+    for s0, e in q1m.prefill_bounds(w):
         c = r[:, s0:e]
         out["per_chunk"].append({"rows": [s0, e], "mean": c.mean().item(), "min": c.min().item(),
                                  "per_head_mean": [round(x, 6) for x in c.mean(1).tolist()]})

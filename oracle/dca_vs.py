@@ -129,8 +129,38 @@ def dca_logits(q_rows: np.ndarray, i_rows: np.ndarray, krot: np.ndarray, js: np.
 # ----------------------------------------------------------------------------------------
 def prefill_chunks(cfg):
     """Yield (s0, e): query rows [s0, e) of each prefill chunk; keys are [0, e)."""
+    if getattr(cfg, "equal_cost_chunks", 0) > 0:
+        yield from equal_cost_chunks(cfg.seq_len, cfg.equal_cost_chunks)
+        return
     for s0 in range(0, cfg.seq_len, cfg.prefill_chunk):
         yield s0, min(cfg.seq_len, s0 + cfg.prefill_chunk)
+
+
+def equal_cost_chunks(n: int, K: int):
+    """Prefill chunks of equal dense attention cost ([P2] 四, pipeline-parallel optimisation,
+    DCPP, Figure 9: chunk sizes follow the attention kernel's cost so that chunks take equal
+    time). READING: the cost unit is one 128 x 128 block of the dense causal mask, so query
+    block b costs b + 1 and the first m blocks cost 1 + 2 + ... + m. Chunk k < K closes at
+    the first block boundary where that cumulative cost reaches k/K of the whole; the last
+    chunk closes at n. A boundary that repeats the previous one is dropped."""
+    nb = -(-n // BLOCK)
+    cum = []                       # cum[i] = cost of blocks 0..i (Python ints: exact)
+    total = 0
+    for b in range(nb):
+        total += b + 1
+        cum.append(total)
+    import bisect
+    cuts = []
+    for k in range(1, K):
+        need = -(-k * total // K)  # ceil(k T / K): cumulative cost the chunk must reach
+        m = bisect.bisect_left(cum, need) + 1
+        if not cuts or m > cuts[-1]:
+            cuts.append(m)
+    rows = [min(n, BLOCK * m) for m in cuts if m < nb] + [n]
+    s0 = 0
+    for e in rows:
+        yield s0, e
+        s0 = e
 
 
 def softmax_rows(l: np.ndarray):

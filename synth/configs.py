@@ -38,6 +38,7 @@ class Workload:
     band_hi: int = 65536
     seed: int = 0
     out_dtype: str = "f32"
+    equal_cost_chunks: int = 0  # K > 0: K prefill chunks of equal dense attention cost
 
     @property
     def dense(self) -> bool:

@@ -403,3 +403,35 @@ def check_recall() -> float:
     return max(float(np.max(np.abs(rec - np.exp(lse_s - lse_d)))),
                float(np.max(np.abs(of.recall_rows(rows, 1, sf) - 1.0))),
                float(max(0.0, np.max(rec) - 1.0)))
+
+
+def check_equal_cost_chunks() -> int:
+    """The equal-cost chunking against the hand-worked fixture and its invariants: chunks
+    tile [0, n) in 128-row blocks, there are at most K, and each chunk's dense cost is within
+    one block row's cost (the largest block's b + 1) of T / K, except that dropped empty
+    chunks merge their share into a neighbour. Returns the number of cases checked."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "equal_cost_chunks.txt")
+    cases = 0
+    for line in open(path):
+        if not line.strip() or line.startswith("#"):
+            continue
+        n, K, *ends = (int(x) for x in line.split())
+        got = [e for _, e in O.equal_cost_chunks(n, K)]
+        assert got == ends, (n, K, got, ends)
+        cases += 1
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        n = int(rng.integers(1, 40000)); K = int(rng.integers(1, 40))
+        ch = list(O.equal_cost_chunks(n, K))
+        nb = -(-n // 128)
+        assert ch[0][0] == 0 and ch[-1][1] == n and len(ch) <= K
+        assert all(a[1] == b[0] for a, b in zip(ch, ch[1:]))
+        assert all(e % 128 == 0 for _, e in ch[:-1]) and all(e > s for s, e in ch)
+        T = nb * (nb + 1) // 2
+        costs = [sum(b + 1 for b in range(s // 128, -(-e // 128))) for s, e in ch]
+        assert sum(costs) == T
+        if len(ch) == K:   # nothing dropped: every chunk is within one block of T / K
+            assert max(abs(c - T / K) for c in costs) <= nb + 1, (n, K, costs)
+        cases += 1
+    return cases

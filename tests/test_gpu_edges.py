@@ -36,6 +36,8 @@ EDGES = [
     BASE.with_(name="last-q-16", vs_last_q=16, vs_force_local=8),
     BASE.with_(name="no-yarn", yarn_s=0.5),
     BASE.with_(name="ragged-many", seq_len=1111, prefill_chunk=384),
+    BASE.with_(name="equal-cost-4", seq_len=1500, equal_cost_chunks=4),
+    BASE.with_(name="equal-cost-dense", seq_len=900, equal_cost_chunks=3, vs_vertical=0, vs_slash=0),
 ]
 
 

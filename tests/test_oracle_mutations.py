@@ -29,7 +29,38 @@ def _all_checks():
     res["force"] = C.check_force_local()
     res["mask"] = C.check_mask_brute_force()
     res["attended"] = C.check_attended_set()
+    res["chunks"] = _passes(C.check_equal_cost_chunks)
     return res
+
+
+def _passes(check) -> bool:
+    try:
+        check()
+        return True
+    except AssertionError:
+        return False
+
+
+def _chunks_variant(cost_of_block, ceil_target=True, drop_repeats=True):
+    def chunks(n, K):
+        nb = -(-n // O.BLOCK)
+        cum, total = [], 0
+        for b in range(nb):
+            total += cost_of_block(b)
+            cum.append(total)
+        import bisect
+        cuts = []
+        for k in range(1, K):
+            need = -(-k * total // K) if ceil_target else k * total // K
+            m = bisect.bisect_left(cum, need) + 1
+            if not drop_repeats or not cuts or m > cuts[-1]:
+                cuts.append(m)
+        rows = [min(n, O.BLOCK * m) for m in cuts if m < nb] + [n]
+        s0 = 0
+        for e in rows:
+            yield s0, e
+            s0 = e
+    return chunks
 
 
 def _rope_sign(x, pos, base):
@@ -151,6 +182,11 @@ MUTATIONS = [
     ("forced local diagonals dropped", "select_head", _select_no_force),
     ("vertical columns left out of the attended set", "attended_mask",
      _attended_without_verticals),
+    ("chunk cost of block b taken as b", "equal_cost_chunks", _chunks_variant(lambda b: b)),
+    ("chunk cost of block b taken as 1", "equal_cost_chunks", _chunks_variant(lambda b: 1)),
+    ("chunk target rounded down", "equal_cost_chunks", _chunks_variant(lambda b: b + 1, ceil_target=False)),
+    ("repeated chunk boundaries kept", "equal_cost_chunks",
+     _chunks_variant(lambda b: b + 1, drop_repeats=False)),
 ]
 
 

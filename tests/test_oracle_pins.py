@@ -76,3 +76,7 @@ def test_attended_set_enumeration():
 
 def test_recall_identity_and_full_budget():
     assert C.check_recall() < 1e-12
+
+
+def test_equal_cost_chunks_fixture_and_invariants():
+    assert C.check_equal_cost_chunks() > 200
