@@ -269,6 +269,35 @@ const char* q1m_last_error(void);
 const char* q1m_version(void);
 
 /* ---------------------------------------------------------------------------------------
+ * Decode
+ * ------------------------------------------------------------------------------------- */
+
+/* Bytes of device scratch q1m_dca_decode needs (the token's query views and the split-KV
+ * partials; independent of the position). 0 on bad input. */
+size_t q1m_dca_decode_scratch_bytes(int n_q_heads, int head_dim);
+
+/* One decode step of the layer ([P2] 四 "Dual Chunk Attention": the token's logits against
+ * every cached key use the same intra / successive / inter remap and YaRN scale as the
+ * prefill; [P2] 三: generation up to 8K tokens after the long context). The token sits at
+ * position pos and attends keys [0, pos], densely.
+ *  - q: [Hq][D], k, v: [Hkv][D] in p->in_dtype: the token's projections (device).
+ *  - k_rot, v16: the fp16 cache [Hkv][ld_tokens][D] (ld_tokens a multiple of 128, > pos).
+ *    Rows [0, pos) hold the earlier tokens' keys rotated at j mod L and their values, as
+ *    q1m_rope_dca_keys or earlier q1m_dca_decode calls write them. The call rotates the
+ *    token's key (position pos mod L), stores it and its value at row pos, and zeroes rows
+ *    (pos, round_up(pos + 1, 32)) of both.
+ *  - table: the RoPE table of q1m_rope_table for (rope_base, dca_chunk, D).
+ *  - out: [Hq][D] in p->out_dtype; lse (nullable): [Hq] fp32, natural log.
+ *  - The budgets and prefill_chunk of p are not used (decode is dense).
+ * Asynchronous on `stream`; fp16 overflow of the token's key, value or query views latches
+ * Q1M_ERR_RANGE (q1m_status_poll). */
+q1m_status q1m_dca_decode(const void* q, const void* k, const void* v, int64_t pos,
+                          uint16_t* k_rot, uint16_t* v16, int64_t ld_tokens, int n_q_heads,
+                          int n_kv_heads, int head_dim, const q1m_params* p, const float* table,
+                          void* out, float* lse, void* scratch, size_t scratch_bytes,
+                          void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * Measurement
  * ------------------------------------------------------------------------------------- */
 
@@ -282,7 +311,8 @@ enum {
   Q1M_STAGE_MASKS = 5,     /* block masks and residual columns        */
   Q1M_STAGE_ATTN = 6,      /* block-sparse attention kernel           */
   Q1M_STAGE_MERGE = 7,     /* LSE merge of the DCA patterns           */
-  Q1M_NUM_STAGES = 8
+  Q1M_STAGE_DECODE = 8,    /* decode attention kernel (q1m_dca_decode) */
+  Q1M_NUM_STAGES = 9
 };
 
 /* Enables (1) or disables (0) per-stage CUDA-event timing inside q1m_dca_sparse_prefill on

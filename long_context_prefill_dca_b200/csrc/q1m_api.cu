@@ -19,6 +19,7 @@
 #include "vs_estimate.cuh"
 #include "attn_tc.cuh"
 #include "lse_merge.cuh"
+#include "decode.cuh"
 
 using namespace q1m;
 
@@ -446,6 +447,68 @@ q1m_status run_merge(const float* o_part, const float* lse_part, int n_parts, in
   return Q1M_OK;
 }
 
+struct DecScratch {
+  size_t qv, o_part, lse_part, total;
+};
+
+DecScratch dec_scratch(int hq, int d) {
+  DecScratch L{};
+  size_t off = 0;
+  L.qv = off; off = align_up(off + (size_t)3 * hq * d * 2);
+  L.o_part = off; off = align_up(off + (size_t)DEC_MAX_SPLIT * hq * d * 4);
+  L.lse_part = off; off = align_up(off + (size_t)DEC_MAX_SPLIT * hq * 4);
+  L.total = off;
+  return L;
+}
+
+template <int D, typename T>
+q1m_status run_decode_d(const T* q, const T* k, const T* v, int64_t pos, uint16_t* k_rot,
+                        uint16_t* v16, int64_t ld_tokens, int hq, int hkv, const q1m_params* p,
+                        const float* table, void* out, float* lse, void* scratch, const Dev& dev,
+                        cudaStream_t st) {
+  const DecScratch SL = dec_scratch(hq, D);
+  const int64_t L = p->dca_chunk - p->local_window;
+  uint16_t* qv = at<uint16_t>(scratch, SL.qv);
+  float* o_part = at<float>(scratch, SL.o_part);
+  float* lse_part = at<float>(scratch, SL.lse_part);
+  const float2* tab = reinterpret_cast<const float2*>(table);
+  const int64_t rows = (pos / DEC_TILE + 1) * DEC_TILE - pos;
+  dec_append_kernel<T><<<blocks_for((int64_t)hkv * rows * (D / 2), 256), 256, 0, st>>>(
+      k, v, hkv, D, pos, L, ld_tokens, tab, k_rot, v16);
+  Q1M_LAUNCHED();
+  dec_queries_kernel<T><<<blocks_for((int64_t)3 * hq * (D / 2), 256), 256, 0, st>>>(
+      q, hq, D, pos, L, p->dca_chunk, tab, view_scale(p, D), qv);
+  Q1M_LAUNCHED();
+  DecArgs a{};
+  a.qv = qv; a.pos = pos; a.L = L; a.n_keys = pos + 1;
+  a.hq = hq; a.G = hq / hkv; a.ld_tokens = ld_tokens;
+  a.n_tiles = (pos + 1 + DEC_TILE - 1) / DEC_TILE;
+  int64_t ns = (dev.sms + hkv - 1) / hkv;
+  const int64_t by_tiles = (a.n_tiles + DEC_WARPS - 1) / DEC_WARPS;   // at least a tile per warp
+  ns = ns < by_tiles ? ns : by_tiles;
+  ns = ns < DEC_MAX_SPLIT ? ns : DEC_MAX_SPLIT;
+  ns = ns < 1 ? 1 : ns;
+  a.tiles_per_split = (a.n_tiles + ns - 1) / ns;
+  a.nsplit = (int)((a.n_tiles + a.tiles_per_split - 1) / a.tiles_per_split);
+  a.o_part = o_part; a.lse_part = lse_part;
+  CUtensorMap mk, mv;
+  Q1M_TRY(make_map(&mk, k_rot, D, (uint64_t)hkv * ld_tokens, 64, DEC_TILE));
+  Q1M_TRY(make_map(&mv, v16, D, (uint64_t)hkv * ld_tokens, 64, DEC_TILE));
+  const size_t smem = sizeof(DecSmem<D>) + 1024;
+  Q1M_CUDA(cudaFuncSetAttribute(dca_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int pr = prof_begin(Q1M_STAGE_DECODE, st);
+  dca_decode_kernel<D><<<dim3(a.nsplit, hkv), 32 * DEC_WARPS, smem, st>>>(mk, mv, a);
+  prof_end(pr, st);
+  Q1M_LAUNCHED();
+  const int grid = blocks_for((int64_t)hq * 32, 256);
+  if (p->out_dtype == Q1M_BF16)
+    dec_merge_kernel<__nv_bfloat16, D><<<grid, 256, 0, st>>>(o_part, lse_part, a.nsplit, hq, (__nv_bfloat16*)out, lse);
+  else
+    dec_merge_kernel<float, D><<<grid, 256, 0, st>>>(o_part, lse_part, a.nsplit, hq, (float*)out, lse);
+  Q1M_LAUNCHED();
+  return Q1M_OK;
+}
+
 }  // namespace
 
 // =============================================================================================
@@ -680,6 +743,40 @@ q1m_status q1m_dca_sparse_prefill_host(const void* q_h, const void* k_h, const v
   Q1M_CUDA(cudaMemcpyAsync(out_h, dout, bo, cudaMemcpyDeviceToHost, st));
   if (lse_h) Q1M_CUDA(cudaMemcpyAsync(lse_h, dlse, (size_t)n * hq * 4, cudaMemcpyDeviceToHost, st));
   return q1m_status_poll(stream);
+}
+
+size_t q1m_dca_decode_scratch_bytes(int hq, int d) {
+  if (hq <= 0 || (d != 64 && d != 128)) return 0;
+  return dec_scratch(hq, d).total;
+}
+
+q1m_status q1m_dca_decode(const void* q, const void* k, const void* v, int64_t pos, uint16_t* k_rot,
+                          uint16_t* v16, int64_t ld_tokens, int hq, int hkv, int d,
+                          const q1m_params* p, const float* table, void* out, float* lse,
+                          void* scratch, size_t scratch_bytes, void* stream) {
+  if (pos < 0) return fail(Q1M_ERR_INVALID, "pos must be >= 0");
+  Q1M_TRY(check_shape(pos + 1, hq, hkv, d, p));
+  if (!q || !k || !v || !k_rot || !v16 || !table || !out || !scratch) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (ld_tokens <= pos || ld_tokens % 128) return fail(Q1M_ERR_INVALID, "ld_tokens must be a multiple of 128 and > pos");
+  if ((int64_t)hkv * ld_tokens >= ((int64_t)1 << 31)) return fail(Q1M_ERR_UNSUPPORTED, "n_kv_heads * ld_tokens too large");
+  if (hq / hkv > 8) return fail(Q1M_ERR_UNSUPPORTED, "decode supports at most 8 Q heads per KV head");
+  if (scratch_bytes < q1m_dca_decode_scratch_bytes(hq, d)) return fail(Q1M_ERR_WORKSPACE, "decode scratch too small");
+  if (reinterpret_cast<uintptr_t>(scratch) & 255) return fail(Q1M_ERR_INVALID, "scratch must be 256-byte aligned");
+  Dev dev;
+  Q1M_TRY(device_info(&dev));
+  cudaStream_t st = S(stream);
+  if (p->in_dtype == Q1M_BF16) {
+    auto* qq = static_cast<const __nv_bfloat16*>(q);
+    auto* kk = static_cast<const __nv_bfloat16*>(k);
+    auto* vv = static_cast<const __nv_bfloat16*>(v);
+    if (d == 128) return run_decode_d<128>(qq, kk, vv, pos, k_rot, v16, ld_tokens, hq, hkv, p, table, out, lse, scratch, dev, st);
+    return run_decode_d<64>(qq, kk, vv, pos, k_rot, v16, ld_tokens, hq, hkv, p, table, out, lse, scratch, dev, st);
+  }
+  auto* qq = static_cast<const float*>(q);
+  auto* kk = static_cast<const float*>(k);
+  auto* vv = static_cast<const float*>(v);
+  if (d == 128) return run_decode_d<128>(qq, kk, vv, pos, k_rot, v16, ld_tokens, hq, hkv, p, table, out, lse, scratch, dev, st);
+  return run_decode_d<64>(qq, kk, vv, pos, k_rot, v16, ld_tokens, hq, hkv, p, table, out, lse, scratch, dev, st);
 }
 
 int64_t q1m_prefill_bounds(int64_t n, const q1m_params* p, int64_t* ends, int64_t max_chunks) {

@@ -30,6 +30,12 @@ __device__ __forceinline__ float load_as_f32<__nv_bfloat16>(const __nv_bfloat16*
   return __bfloat162float(*p);
 }
 
+// The rotate-half pair (x1, x2) by the angle with (cos, sin) = cs, with one fixed rounding
+// (explicit fused multiply-adds), so that every kernel that rotates the same values (the
+// prefill's keys and views, the decode step's) produces the same bits.
+__device__ __forceinline__ float rot_lo(float x1, float x2, float2 cs) { return __fmaf_rn(x1, cs.x, -(x2 * cs.y)); }
+__device__ __forceinline__ float rot_hi(float x1, float x2, float2 cs) { return __fmaf_rn(x2, cs.x, x1 * cs.y); }
+
 __device__ __forceinline__ uint16_t to_f16_checked(float x) {
   if (!(fabsf(x) <= 65504.f)) latch(Q1M_ERR_RANGE);   // also catches NaN
   return __half_as_ushort(__float2half_rn(x));
@@ -64,8 +70,8 @@ __global__ void rope_keys_kernel(const T* __restrict__ k, const T* __restrict__ 
   const float x1 = load_as_f32(k + src + f), x2 = load_as_f32(k + src + f + hd);
   const float2 cs = table[(j % L) * hd + f];
   const int64_t dst = ((int64_t)g * ld_tokens + j) * d;
-  k_rot[dst + f] = to_f16_checked(x1 * cs.x - x2 * cs.y);
-  k_rot[dst + f + hd] = to_f16_checked(x2 * cs.x + x1 * cs.y);
+  k_rot[dst + f] = to_f16_checked(rot_lo(x1, x2, cs));
+  k_rot[dst + f + hd] = to_f16_checked(rot_hi(x1, x2, cs));
   v16[dst + f] = to_f16_checked(load_as_f32(v + src + f));
   v16[dst + f + hd] = to_f16_checked(load_as_f32(v + src + f + hd));
 }
@@ -104,8 +110,8 @@ __global__ void rope_queries_kernel(const T* __restrict__ q, int64_t s0, int64_t
     uint16_t y1 = 0, y2 = 0;
     if (i < e) {
       const float2 cs = table[dca_query_pos(i, x, L, c) * hd + f];
-      y1 = to_f16_checked(x1 * cs.x - x2 * cs.y);
-      y2 = to_f16_checked(x2 * cs.x + x1 * cs.y);
+      y1 = to_f16_checked(rot_lo(x1, x2, cs));
+      y2 = to_f16_checked(rot_hi(x1, x2, cs));
     }
     qv[dst + f] = y1;
     qv[dst + f + hd] = y2;
@@ -145,8 +151,8 @@ __global__ void est_queries_kernel(const T* __restrict__ q, int64_t r_lo, int64_
       const float x1 = load_as_f32(q + src + f) * scale;
       const float x2 = load_as_f32(q + src + f + hd) * scale;
       const float2 cs = table[dca_query_pos(i, view, L, c) * hd + f];
-      y1 = to_f16_checked(x1 * cs.x - x2 * cs.y);
-      y2 = to_f16_checked(x2 * cs.x + x1 * cs.y);
+      y1 = to_f16_checked(rot_lo(x1, x2, cs));
+      y2 = to_f16_checked(rot_hi(x1, x2, cs));
     }
   }
   const int64_t dst = (((int64_t)cls * hkv + g) * m_pad + m) * d;

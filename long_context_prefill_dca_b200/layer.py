@@ -128,3 +128,14 @@ class Stages:
         w = self.w
         q1m.lse_merge(self.o_part, self.lse_part, 3, self.ld_rows, s0, e, w.seq_len,
                       w.n_q_heads, w.head_dim, self.p.out_dtype, self.p, out, lse)
+
+    def decode(self, q_tok, k_tok, v_tok, pos, out, lse=None):
+        """One decode step: the token at `pos` (q [Hq][D], k, v [Hkv][D]) is appended to the
+        cache and attends keys [0, pos]; out [Hq][D], lse [Hq] (natural log)."""
+        w = self.w
+        nb = q1m.dca_decode_scratch_bytes(w.n_q_heads, w.head_dim)
+        if getattr(self, "_dec_scratch", None) is None or self._dec_scratch.numel() < nb:
+            self._dec_scratch = torch.empty(nb, dtype=torch.uint8, device=self.dev)
+        q1m.dca_decode(q_tok, k_tok, v_tok, pos, self.k_rot, self.v16, self.ld_tokens,
+                       w.n_q_heads, w.n_kv_heads, w.head_dim, self.p, self.table, out, lse,
+                       self._dec_scratch, nb)

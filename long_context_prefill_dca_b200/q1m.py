@@ -66,6 +66,9 @@ SIGNATURES = {
                               PP, c_vp, c_vp, c_vp]),
     "q1m_attention_recall": (c_int, [c_vp, c_vp, c_i64, c_vp, c_vp]),
     "q1m_prefill_bounds": (c_i64, [c_i64, PP, c_vp, c_i64]),
+    "q1m_dca_decode_scratch_bytes": (c_size, [c_int, c_int]),
+    "q1m_dca_decode": (c_int, [c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_int, c_int, c_int, PP,
+                               c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
     "q1m_status_poll": (c_int, [c_vp]),
     "q1m_last_error": (ctypes.c_char_p, []),
     "q1m_version": (ctypes.c_char_p, []),
@@ -221,6 +224,17 @@ def attention_recall(lse_sparse, lse_dense, recall, stream=None) -> None:
           stream_handle(stream))
 
 
+def dca_decode_scratch_bytes(hq, d) -> int:
+    return int(library().q1m_dca_decode_scratch_bytes(hq, d))
+
+
+def dca_decode(q, k, v, pos, k_rot, v16, ld_tokens, hq, hkv, d, p, table, out, lse, scratch,
+               scratch_bytes, stream=None) -> None:
+    _call("q1m_dca_decode", ptr(q), ptr(k), ptr(v), int(pos), ptr(k_rot), ptr(v16), int(ld_tokens),
+          hq, hkv, d, ctypes.byref(p), ptr(table), ptr(out), ptr(lse), ptr(scratch),
+          int(scratch_bytes), stream_handle(stream))
+
+
 def prefill_bounds(w) -> list[tuple[int, int]]:
     """(s0, e) of every prefill chunk of workload w, as the library's driver loop runs them
     (host computation; no GPU needed)."""
@@ -256,7 +270,7 @@ def selftest_wait_timeout(cycles: int, stream=None) -> int:
     return library().q1m_selftest_wait_timeout(cycles, stream_handle(stream))
 
 
-STAGES = ["table", "keys", "queries", "estimate", "select", "masks", "attn", "merge"]
+STAGES = ["table", "keys", "queries", "estimate", "select", "masks", "attn", "merge", "decode"]
 
 
 def profile_enable(on: bool = True) -> None:

@@ -353,6 +353,16 @@ class Oracle:
         p, lse = softmax_rows(l)
         return p @ self.v[: imax + 1, h // self.cfg.group, :], lse
 
+    def decode_row(self, pos: int, h: int):
+        """Decode step of the token at `pos`: out and lse of head h over keys [0, pos] with
+        the DCA logits, densely ([P2] 四 "Dual Chunk Attention"; [P2] 三: generation after the
+        long context). Equals row pos of the dense prefill by definition."""
+        js = np.arange(pos + 1)
+        l = dca_logits(self.q_rows(np.array([pos]), h), np.array([pos]),
+                       self.krot(h // self.cfg.group)[: pos + 1], js, self.cfg)
+        p, lse = softmax_rows(l)
+        return (p @ self.v[: pos + 1, h // self.cfg.group, :])[0], float(lse[0])
+
     def recall_rows(self, rows: np.ndarray, h: int, sel: ChunkSelection) -> np.ndarray:
         """Share of the dense softmax mass of each row that its attended set A(i) keeps
         ([P2] 四 稀疏注意力机制: sparsity refinement limits the accuracy loss)."""

@@ -435,3 +435,28 @@ def check_equal_cost_chunks() -> int:
             assert max(abs(c - T / K) for c in costs) <= nb + 1, (n, K, costs)
         cases += 1
     return cases
+
+
+def check_decode_row() -> float:
+    """The decode step against pair-by-pair brute force (independently worded relative
+    positions, complex-arithmetic RoPE) over every key j <= pos, for positions on both sides
+    of DCA chunk boundaries, and V = 1 giving out = 1."""
+    cfg = tiny(yarn_s=3.0, n_q_heads=3, n_kv_heads=1)
+    q, k, v = rand_qkv(cfg, 9)
+    orc = O.Oracle(q, k, v, cfg)
+    scale = O.yarn_inv_t(cfg.yarn_s) / math.sqrt(cfg.head_dim)
+    L = O.dca_len(cfg)
+    err = 0.0
+    for pos in (0, 1, L - 1, L, 2 * L - 1, 2 * L, 2 * L + 5, cfg.seq_len - 1):
+        for h in range(cfg.n_q_heads):
+            got, lse = orc.decode_row(pos, h)
+            lg = np.array([brute_logit(q[pos, h], k[j, 0], brute_relative(pos, j, cfg.dca_chunk,
+                                                                          cfg.local_window),
+                                       cfg.rope_base, scale) for j in range(pos + 1)])
+            mx = lg.max()
+            w = np.exp(lg - mx)
+            ref = (w[:, None] * v[: pos + 1, 0, :]).sum(0) / w.sum()
+            err = max(err, float(np.max(np.abs(got - ref))), abs(lse - (mx + math.log(w.sum()))))
+    ones = O.Oracle(q, k, np.ones_like(v), cfg)
+    err = max(err, float(np.max(np.abs(ones.decode_row(cfg.seq_len - 1, 1)[0] - 1.0))))
+    return err

@@ -75,3 +75,24 @@ def test_workspace_sizes_monotone(lib):
     small = q1m.workspace_bytes(C.L7B_128K.seq_len, 28, 4, 128, q1m.params(C.L7B_128K))
     big = q1m.workspace_bytes(C.L7B_1M.seq_len, 28, 4, 128, q1m.params(C.L7B_1M))
     assert 0 < small < big < 40 * 2**30
+
+
+def test_decode_validates_before_launch():
+    """q1m_dca_decode rejects bad arguments on the host, before touching the device."""
+    import ctypes
+    from long_context_prefill_dca_b200 import q1m
+    from synth import configs as C
+    lib = q1m.library()
+    w = C.SMALL_SPARSE.with_(vs_vertical=0, vs_slash=0)
+    p = q1m.params(w)
+    nb = q1m.dca_decode_scratch_bytes(w.n_q_heads, w.head_dim)
+    assert nb > 0 and q1m.dca_decode_scratch_bytes(4, 96) == 0
+    args = lambda pos, ld, hq, hkv, d, sc: (1, 1, 1, pos, 256, 256, ld, hq, hkv, d, ctypes.byref(p), 256,
+                                            256, None, 256, sc, None)
+    assert lib.q1m_dca_decode(*args(-1, 1024, 4, 2, 128, nb)) == -1            # bad position
+    assert lib.q1m_dca_decode(*args(1024, 1024, 4, 2, 128, nb)) == -1          # pos beyond the cache
+    assert lib.q1m_dca_decode(*args(10, 1000, 4, 2, 128, nb)) == -1            # ld_tokens % 128
+    assert lib.q1m_dca_decode(*args(10, 1024, 16, 1, 128, nb)) == -2           # G > 8
+    assert lib.q1m_dca_decode(*args(10, 1024, 4, 2, 128, nb - 1)) == -3        # scratch too small
+    assert lib.q1m_dca_decode(None, 1, 1, 10, 256, 256, 1024, 4, 2, 128, ctypes.byref(p), 256, 256,
+                              None, 256, nb, None) == -1                       # NULL pointer

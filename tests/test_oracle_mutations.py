@@ -30,6 +30,7 @@ def _all_checks():
     res["mask"] = C.check_mask_brute_force()
     res["attended"] = C.check_attended_set()
     res["chunks"] = _passes(C.check_equal_cost_chunks)
+    res["decode"] = C.check_decode_row() < 1e-10
     return res
 
 

@@ -80,3 +80,7 @@ def test_recall_identity_and_full_budget():
 
 def test_equal_cost_chunks_fixture_and_invariants():
     assert C.check_equal_cost_chunks() > 200
+
+
+def test_decode_row_brute_force():
+    assert C.check_decode_row() < 1e-10
