@@ -66,6 +66,10 @@ def parse():
     ap.add_argument("--out-dtype", default="bf16", choices=["bf16", "f32"])
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="with N > 1 GPUs: independent replicas of the layer (weak scaling), or "
+                         "the layer's KV-head groups split over the ranks (strong scaling; no "
+                         "exchange inside attention, an all-gather of the output after it)")
     ap.add_argument("--equal-cost-chunks", type=int, default=0,
                     help="K > 0: K prefill chunks of equal dense attention cost instead of the "
                          "workload's fixed prefill chunk")
@@ -84,8 +88,20 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
 
 
 def job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
-    """Whole-job throughput: the work of every rank over the slowest rank's step time."""
+    """Whole-job throughput of replicas: the work of every rank over the slowest rank's step
+    time."""
     return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
+def sum_over_ranks(value: float, world: int, device=None) -> float:
+    """The sum of every rank's value (all ranks call this in the same order)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
 
 
 def peaks():
@@ -301,8 +317,13 @@ def main():
     w = C.BY_NAME[args.workload].with_(out_dtype=args.out_dtype,
                                         equal_cost_chunks=args.equal_cost_chunks)
     q1m.library()
-
+    sharded = args.shard == "heads" and world > 1
+    w_full = w
     x = I.generate(w)
+    if sharded:
+        from long_context_prefill_dca_b200 import parallel as P
+        x = P.shard_inputs(x, w, rank, world)
+        w = P.shard_workload(w, rank, world)
     g = {k: t.to(device) for k, t in x.items()}
     pairs, density, per_chunk = attended_pairs(w, g, device)
     flops = 4.0 * w.head_dim * pairs
@@ -347,7 +368,20 @@ def main():
     clk = clocks.stop()
     q1m.check_status(stream)
     ms_step = max_over_ranks(ev0.elapsed_time(ev1), world, device) / args.steps
-    value = job_tflops(flops, world, ms_step)
+    job_flops = sum_over_ranks(flops, world, device)   # replicas: world x flops
+    value = job_flops / (ms_step * 1e-3) / 1e12
+    allgather_ms = None
+    if sharded:
+        # the only collective of the sharded layer, after attention: out over heads
+        from long_context_prefill_dca_b200 import parallel as P
+        dist.barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        full = P.gather_heads(out, world)
+        a1.record(stream)
+        torch.cuda.synchronize(device)
+        allgather_ms = max_over_ranks(a0.elapsed_time(a1), world, device)
+        del full
 
     # e2e: the same layer through the host-buffer entry point, copies included
     e2e = None
@@ -369,7 +403,7 @@ def main():
         torch.cuda.synchronize(device)
         ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, device)
         h2d = sum(v.numel() * v.element_size() for v in pin.values())
-        e2e = {"value": job_tflops(flops, world, ms_e2e), "unit": UNIT,
+        e2e = {"value": job_flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": args.e2e_steps}
         del hl, pin, out_h
@@ -410,10 +444,11 @@ def main():
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
             "dtype": "f16", "data": "synthetic (seeded N(0,1) + planted sinks/bands, bf16)",
-            "config": {"workload": w.name, "seq_len": w.seq_len, "n_q_heads": w.n_q_heads,
-                       "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+            "config": {"workload": w.name, "seq_len": w.seq_len, "n_q_heads": w_full.n_q_heads,
+                       "n_kv_heads": w_full.n_kv_heads, "head_dim": w.head_dim,
+                       "heads_per_rank": [w.n_q_heads, w.n_kv_heads],
                        "dca_chunk": w.dca_chunk, "local_window": w.local_window,
                        "yarn_s": w.yarn_s, "prefill_chunk": w.prefill_chunk,
                        "chunking": (f"equal-cost x{w.equal_cost_chunks}" if w.equal_cost_chunks
@@ -421,9 +456,11 @@ def main():
                        "prefill_chunks": [list(b) for b in q1m.prefill_bounds(w)],
                        "vs_budget": [w.vs_vertical, w.vs_slash], "inputs": "bf16",
                        "mma": "f16 x f16 -> f32", "out": args.out_dtype,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "parallelism": (f"KV-head groups split over {world} GPUs" if sharded else
+                                       f"replicas x{world}" if world > 1 else "single GPU"),
+                       "allgather_ms": allgather_ms,
                        "l2": "inputs (9.6 GB) far larger than L2 (126 MB); no flush",
-                       "attended_pairs": pairs, "block_density": density,
+                       "attended_pairs": job_flops / (4.0 * w.head_dim), "block_density": density,
                        "ms_per_layer": ms_step},
             "roofline": roofline, "estimator": estimator, "stages": stages,
             "cpu_baseline": cpu, "e2e": e2e,

@@ -28,7 +28,9 @@ def _rank(rank, world, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
     ms = [120.0, 95.0][rank]               # rank 0 is the slower one
     slow = bench.max_over_ranks(ms, world)
-    q.put((rank, slow, bench.job_tflops(1e15, world, slow)))
+    # head-sharded runs: each rank counts its own shard's work; the job sums them
+    shard_flops = [3e14, 5e14][rank]
+    q.put((rank, slow, bench.job_tflops(1e15, world, slow), bench.sum_over_ranks(shard_flops, world)))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -45,15 +47,17 @@ def test_max_over_ranks_and_job_throughput_gloo():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, slow, tf in res:
+    for rank, slow, tf, total in res:
         assert slow == 120.0
         assert tf == pytest.approx(1e15 * 2 / 0.120 / 1e12)
+        assert total == pytest.approx(8e14)
 
 
 def test_single_rank_passthrough():
     import bench
     assert bench.max_over_ranks(7.5, 1) == 7.5
     assert bench.job_tflops(2e12, 1, 1000.0) == pytest.approx(2.0)
+    assert bench.sum_over_ranks(3.5, 1) == 3.5
 
 
 def test_reference_arm_silent_on_other_ranks():
