@@ -46,7 +46,9 @@ typedef enum {
   Q1M_ERR_WORKSPACE = -3,    /* workspace too small                                        */
   Q1M_ERR_CUDA = -4,         /* a CUDA runtime call failed                                 */
   Q1M_ERR_TIMEOUT = -5,      /* a device-side bounded wait ran out (latched on the device) */
-  Q1M_ERR_RANGE = -6         /* fp16 overflow in the rotation stage, or a NaN score        */
+  Q1M_ERR_RANGE = -6,        /* fp16 overflow in the rotation stage, or a NaN score        */
+  Q1M_ERR_CHECK = -7         /* debug mode: a workspace guard region was overwritten or an
+                              * index list is malformed (q1m_set_debug)                      */
 } q1m_status;
 
 typedef enum { Q1M_BF16 = 0, Q1M_F32 = 1 } q1m_dtype;
@@ -105,6 +107,20 @@ q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, v
                                   float* lse, int64_t seq_len, int n_q_heads, int n_kv_heads,
                                   int head_dim, const q1m_params* p, void* workspace,
                                   size_t workspace_bytes, void* stream);
+
+/* The layer restricted to prefill chunks [first_chunk, last_chunk) (chunk numbers as
+ * q1m_prefill_bounds lists them; last_chunk past the end means "to the end"): a prefill
+ * resumed at chunk granularity. Chunk c attends the rotated keys of chunks 0..c, which live
+ * in the workspace, so chunks before first_chunk must have run on the same workspace (same
+ * shapes and params) with nothing else written to it in between; the rows of out and lse
+ * of the chunks that run are written, the others are left as they are. Running [0, a) and
+ * then [a, end) gives the same result, bit for bit, as one q1m_dca_sparse_prefill call
+ * (which is this call with [0, end)). */
+q1m_status q1m_dca_sparse_prefill_chunks(const void* q, const void* k, const void* v, void* out,
+                                         float* lse, int64_t seq_len, int n_q_heads,
+                                         int n_kv_heads, int head_dim, const q1m_params* p,
+                                         int64_t first_chunk, int64_t last_chunk,
+                                         void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bytes of device workspace q1m_dca_sparse_prefill_host needs (staging for q, k, v, out
  * and lse plus q1m_workspace_bytes). */
@@ -296,6 +312,27 @@ q1m_status q1m_dca_decode(const void* q, const void* k, const void* v, int64_t p
                           int n_kv_heads, int head_dim, const q1m_params* p, const float* table,
                           void* out, float* lse, void* scratch, size_t scratch_bytes,
                           void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Debug mode
+ * ------------------------------------------------------------------------------------- */
+
+/* Debug mode for the whole process (initially on when the environment variable Q1M_DEBUG is
+ * set to a non-zero value). In debug mode q1m_dca_sparse_prefill(_chunks) lays out its
+ * workspace with a 4 KiB guard region after every buffer (so q1m_workspace_bytes grows:
+ * query it after switching), fills the guards with a pattern at the start of each call,
+ * checks every guard after each stage and validates the selected index lists (ascending,
+ * inside [0, e), the forced diagonals present) and the block counts after the mask stage.
+ * A failed check latches Q1M_ERR_CHECK, which q1m_status_poll returns with the failing
+ * guard or list in q1m_last_error. Results are unchanged; the checks cost time. */
+q1m_status q1m_set_debug(int on);
+int q1m_debug_enabled(void);
+
+/* Test hook of the debug mode: on the next layer call, right after the given stage
+ * (Q1M_STAGE_*) of the first prefill chunk, the library overwrites one byte of the first
+ * guard region from the host side (cudaMemsetAsync), so that the following check reports
+ * Q1M_ERR_CHECK. -1 disarms it. Has no effect outside debug mode. */
+q1m_status q1m_debug_inject(int stage);
 
 /* ---------------------------------------------------------------------------------------
  * Measurement

@@ -5,8 +5,10 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstdint>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <atomic>
 #include <mutex>
@@ -234,11 +236,73 @@ EstLayout est_layout(int64_t e, int hq, int hkv, int d) {
 }
 
 // ---- whole-layer workspace layout ---------------------------------------------------------
+// ---- debug mode: guard regions after every workspace buffer, index-list validation -------
+constexpr size_t GUARD_BYTES = 4096;
+constexpr uint32_t GUARD_WORD = 0xA5A5A5A5u;
+constexpr int MAX_GUARDS = 32;
+std::atomic<int> g_debug{-1};
+std::atomic<int> g_inject{-1};
+
+bool debug_on() {
+  int v = g_debug.load();
+  if (v < 0) {
+    const char* e = std::getenv("Q1M_DEBUG");
+    v = (e && *e && std::strcmp(e, "0") != 0) ? 1 : 0;
+    g_debug.store(v);
+  }
+  return v == 1;
+}
+
+__device__ int g_check_info = -1;   // first failing guard (0..) or list check (1000 + kind)
+
+struct GuardSet {
+  uint64_t off[MAX_GUARDS];
+  int n;
+};
+
+__global__ void guard_check_kernel(const uint8_t* __restrict__ base, GuardSet gs) {
+  const int gi = blockIdx.x;
+  if (gi >= gs.n) return;
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(base + gs.off[gi]);
+  for (int i = threadIdx.x; i < (int)(GUARD_BYTES / 4); i += blockDim.x)
+    if (w[i] != GUARD_WORD) { atomicCAS(&g_check_info, -1, gi); latch(Q1M_ERR_CHECK); }
+}
+
+// One thread per head: V ascending in [0, e); S ascending in [0, e) starting with the forced
+// diagonals 0 .. fl - 1; then, per (head, query block), block counts within the key-block
+// count and residual columns ascending in [0, e).
+__global__ void index_check_kernel(const int32_t* __restrict__ V, int nv, const int32_t* __restrict__ Sx,
+                                   int ns, int64_t e, int hq, int fl, const int32_t* __restrict__ cnt,
+                                   const int32_t* __restrict__ resid, int nqb, int nvcap, int64_t nkb) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= hq) return;
+  auto bad = [](int kind) { atomicCAS(&g_check_info, -1, 1000 + kind); latch(Q1M_ERR_CHECK); };
+  for (int i = 0; i < nv; ++i) {
+    const int64_t c = V[(int64_t)h * nv + i];
+    if (c < 0 || c >= e || (i > 0 && c <= V[(int64_t)h * nv + i - 1])) { bad(1); return; }
+  }
+  for (int i = 0; i < ns; ++i) {
+    const int64_t o = Sx[(int64_t)h * ns + i];
+    if (o < 0 || o >= e || (i > 0 && o <= Sx[(int64_t)h * ns + i - 1])) { bad(2); return; }
+    if (i < fl && i < e && o != i) { bad(3); return; }
+  }
+  for (int b = 0; b < nqb; ++b) {
+    const int32_t* c = cnt + ((int64_t)h * nqb + b) * 8;
+    if (c[0] < 0 || c[1] < 0 || c[2] < 0 || c[0] + c[1] + c[2] > nkb) { bad(4); return; }
+    const int nres = c[6];
+    if (nres < 0 || nres > nvcap || c[3] + c[4] + c[5] != nres) { bad(5); return; }
+    const int32_t* r = resid + ((int64_t)h * nqb + b) * nvcap;
+    for (int i = 0; i < nres; ++i)
+      if (r[i] < 0 || r[i] >= e || (i > 0 && r[i] <= r[i - 1])) { bad(6); return; }
+  }
+}
+
 struct Layout {
   int64_t ld_tokens, ld_rows, nqb_max, nkw_max;
   int nv, ns;
   size_t table, k_rot, v16, qv, o_part, lse_part, units, vert, slash, est, V, Sx, mask, resid,
       cnt, total;
+  GuardSet guards{};
 };
 
 Layout layout(int64_t n, int hq, int hkv, int d, const q1m_params* p) {
@@ -250,7 +314,13 @@ Layout layout(int64_t n, int hq, int hkv, int d, const q1m_params* p) {
   L.nv = (int)(p->vs_vertical < n ? p->vs_vertical : n);
   L.ns = (int)(p->vs_slash < n ? p->vs_slash : n);
   size_t off = 0;
-  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+  const bool dbg = debug_on();
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes);
+    if (dbg && L.guards.n < MAX_GUARDS) { L.guards.off[L.guards.n++] = off; off += GUARD_BYTES; }
+    return o;
+  };
   L.table = take((size_t)p->dca_chunk * (d / 2) * sizeof(float2));
   L.k_rot = take((size_t)hkv * L.ld_tokens * d * 2);
   L.v16 = take((size_t)hkv * L.ld_tokens * d * 2);
@@ -276,6 +346,18 @@ template <typename T>
 T* at(void* base, size_t off) { return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off); }
 
 int blocks_for(int64_t n, int threads) { return (int)((n + threads - 1) / threads); }
+
+// Debug mode: checks every guard after `stage` (and first plays the armed injection, once).
+q1m_status debug_after(const Layout& L, void* ws, int stage, bool first_chunk, cudaStream_t st) {
+  if (L.guards.n == 0) return Q1M_OK;
+  if (first_chunk && g_inject.load() == stage) {
+    g_inject.store(-1);
+    Q1M_CUDA(cudaMemsetAsync(at<uint8_t>(ws, L.guards.off[0]), 0, 1, st));
+  }
+  guard_check_kernel<<<L.guards.n, 256, 0, st>>>(static_cast<const uint8_t*>(ws), L.guards);
+  Q1M_LAUNCHED();
+  return Q1M_OK;
+}
 
 // ---- stage launchers (arguments already validated) ------------------------------------------
 q1m_status run_rope_table(float* table, int64_t n_pos, int d, double base, cudaStream_t st) {
@@ -654,7 +736,17 @@ q1m_status q1m_lse_merge(const float* o_part, const float* lse_part, int n_parts
 q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, void* out,
                                   float* lse, int64_t n, int hq, int hkv, int d,
                                   const q1m_params* p, void* ws, size_t ws_bytes, void* stream) {
+  return q1m_dca_sparse_prefill_chunks(q, k, v, out, lse, n, hq, hkv, d, p, 0, INT64_MAX, ws,
+                                       ws_bytes, stream);
+}
+
+q1m_status q1m_dca_sparse_prefill_chunks(const void* q, const void* k, const void* v, void* out,
+                                         float* lse, int64_t n, int hq, int hkv, int d,
+                                         const q1m_params* p, int64_t first_chunk,
+                                         int64_t last_chunk, void* ws, size_t ws_bytes,
+                                         void* stream) {
   Q1M_TRY(check_shape(n, hq, hkv, d, p));
+  if (first_chunk < 0 || last_chunk < first_chunk) return fail(Q1M_ERR_INVALID, "bad chunk range");
   if (!q || !k || !v || !out || !ws) return fail(Q1M_ERR_INVALID, "NULL pointer");
   if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(Q1M_ERR_INVALID, "workspace must be 256-byte aligned");
   const Layout L = layout(n, hq, hkv, d, p);
@@ -670,9 +762,13 @@ q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, v
   float* lse_part = at<float>(ws, L.lse_part);
   int32_t* units = at<int32_t>(ws, L.units);
   const int64_t Ld = p->dca_chunk - p->local_window;
+  // debug mode: guard regions get their pattern at the start of every call
+  for (int gi = 0; gi < L.guards.n; ++gi)
+    Q1M_CUDA(cudaMemsetAsync(at<uint8_t>(ws, L.guards.off[gi]), 0xA5, GUARD_BYTES, st));
   int pr = prof_begin(Q1M_STAGE_TABLE, st);
   Q1M_TRY(run_rope_table(table, p->dca_chunk, d, p->rope_base, st));
   prof_end(pr, st);
+  Q1M_TRY(debug_after(L, ws, Q1M_STAGE_TABLE, true, st));
   if (L.ld_tokens > n) {
     // zero the padded key rows once so tiles past the end read finite values
     for (int g = 0; g < hkv; ++g) {
@@ -680,14 +776,18 @@ q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, v
       Q1M_CUDA(cudaMemsetAsync(v16 + ((int64_t)g * L.ld_tokens + n) * d, 0, (size_t)(L.ld_tokens - n) * d * 2, st));
     }
   }
-  int64_t s0 = 0;
-  for (const int64_t e : chunk_ends(n, p)) {
+  const std::vector<int64_t> ends = chunk_ends(n, p);
+  for (int64_t ci = first_chunk; ci < (int64_t)ends.size() && ci < last_chunk; ++ci) {
+    const int64_t s0 = ci == 0 ? 0 : ends[ci - 1], e = ends[ci];
+    const bool first = ci == first_chunk;
     pr = prof_begin(Q1M_STAGE_KEYS, st);
     Q1M_TRY(run_rope_keys(k, v, s0, e, hkv, d, p, table, k_rot, v16, L.ld_tokens, st));
     prof_end(pr, st);
+    Q1M_TRY(debug_after(L, ws, Q1M_STAGE_KEYS, first, st));
     pr = prof_begin(Q1M_STAGE_QUERIES, st);
     Q1M_TRY(run_rope_queries(q, s0, e, hq, d, p, table, qv, L.ld_rows, st));
     prof_end(pr, st);
+    Q1M_TRY(debug_after(L, ws, Q1M_STAGE_QUERIES, first, st));
     const uint32_t* mask = nullptr;
     const int32_t *resid = nullptr, *cnt = nullptr;
     if (sparse(p)) {
@@ -699,22 +799,34 @@ q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, v
       if (d == 128) Q1M_TRY(run_estimate_d<128>(q, k_rot, L.ld_tokens, s0, e, hq, hkv, p, table, vert, slash, L.ld_tokens, at<void>(ws, L.est), dev, st));
       else Q1M_TRY(run_estimate_d<64>(q, k_rot, L.ld_tokens, s0, e, hq, hkv, p, table, vert, slash, L.ld_tokens, at<void>(ws, L.est), dev, st));
       prof_end(pr, st);
+      Q1M_TRY(debug_after(L, ws, Q1M_STAGE_ESTIMATE, first, st));
       pr = prof_begin(Q1M_STAGE_SELECT, st);
       Q1M_TRY(run_select(vert, slash, L.ld_tokens, e, hq, p, V, Sx, st));
       prof_end(pr, st);
+      Q1M_TRY(debug_after(L, ws, Q1M_STAGE_SELECT, first, st));
       pr = prof_begin(Q1M_STAGE_MASKS, st);
       Q1M_TRY(run_masks(V, Sx, s0, e, hq, p, at<uint32_t>(ws, L.mask), at<int32_t>(ws, L.resid), at<int32_t>(ws, L.cnt), st));
       prof_end(pr, st);
+      Q1M_TRY(debug_after(L, ws, Q1M_STAGE_MASKS, first, st));
+      if (L.guards.n > 0) {
+        const int nv_e = (int)(p->vs_vertical < e ? p->vs_vertical : e);
+        const int ns_e = (int)(p->vs_slash < e ? p->vs_slash : e);
+        index_check_kernel<<<blocks_for(hq, 32), 32, 0, st>>>(
+            V, nv_e, Sx, ns_e, e, hq, p->vs_force_local, at<int32_t>(ws, L.cnt), at<int32_t>(ws, L.resid),
+            (int)((e - s0 + 127) / 128), nv_e, (e + 127) / 128);
+        Q1M_LAUNCHED();
+      }
       mask = at<uint32_t>(ws, L.mask);
       resid = at<int32_t>(ws, L.resid);
       cnt = at<int32_t>(ws, L.cnt);
     }
     if (d == 128) Q1M_TRY(run_attn_d<128>(qv, L.ld_rows, k_rot, v16, L.ld_tokens, mask, resid, cnt, s0, e, hq, hkv, p, o_part, lse_part, units, dev, st));
     else Q1M_TRY(run_attn_d<64>(qv, L.ld_rows, k_rot, v16, L.ld_tokens, mask, resid, cnt, s0, e, hq, hkv, p, o_part, lse_part, units, dev, st));
+    Q1M_TRY(debug_after(L, ws, Q1M_STAGE_ATTN, first, st));
     pr = prof_begin(Q1M_STAGE_MERGE, st);
     Q1M_TRY(run_merge(o_part, lse_part, 3, L.ld_rows, s0, e, n, hq, d, p->out_dtype, Ld, out, lse, st));
     prof_end(pr, st);
-    s0 = e;
+    Q1M_TRY(debug_after(L, ws, Q1M_STAGE_MERGE, first, st));
   }
   return Q1M_OK;
 }
@@ -796,10 +908,32 @@ q1m_status q1m_status_poll(void* stream) {
   int st = 0;
   Q1M_CUDA(cudaMemcpyFromSymbol(&st, g_status, sizeof(int)));
   if (st != 0) {
-    const int zero = 0;
+    const int zero = 0, none = -1;
+    int info = -1;
+    Q1M_CUDA(cudaMemcpyFromSymbol(&info, g_check_info, sizeof(int)));
     Q1M_CUDA(cudaMemcpyToSymbol(g_status, &zero, sizeof(int)));
+    Q1M_CUDA(cudaMemcpyToSymbol(g_check_info, &none, sizeof(int)));
+    if (st == Q1M_ERR_CHECK) {
+      static const char* lists[] = {"", "vertical columns", "slash offsets", "forced diagonals",
+                                    "block counts", "residual counts", "residual columns"};
+      if (info >= 1000 && info < 1007) return fail(Q1M_ERR_CHECK, "debug check: malformed %s", lists[info - 1000]);
+      return fail(Q1M_ERR_CHECK, "debug check: workspace guard region %d overwritten", info);
+    }
     return fail((q1m_status)st, st == Q1M_ERR_TIMEOUT ? "a device-side wait ran out" : "device-side range/NaN check failed");
   }
+  return Q1M_OK;
+}
+
+q1m_status q1m_set_debug(int on) {
+  g_debug.store(on ? 1 : 0);
+  return Q1M_OK;
+}
+
+int q1m_debug_enabled(void) { return debug_on() ? 1 : 0; }
+
+q1m_status q1m_debug_inject(int stage) {
+  if (stage < -1 || stage >= Q1M_NUM_STAGES) return fail(Q1M_ERR_INVALID, "bad stage %d", stage);
+  g_inject.store(stage);
   return Q1M_OK;
 }
 

@@ -34,6 +34,15 @@ class Layer:
                                w.head_dim, self.p, self.ws, self.ws_bytes, stream)
         return out
 
+    def chunks(self, q, k, v, first, last, out, lse=None, stream=None):
+        """Prefill chunks [first, last) only, on this layer's workspace: a prefill resumed at
+        chunk granularity (chunks before `first` must have run on this layer already)."""
+        w = self.w
+        q1m.dca_sparse_prefill_chunks(q, k, v, out, lse, w.seq_len, w.n_q_heads, w.n_kv_heads,
+                                      w.head_dim, self.p, first, last, self.ws, self.ws_bytes,
+                                      stream)
+        return out
+
 
 class HostLayer:
     """The layer from host (pinned) buffers through q1m_dca_sparse_prefill_host."""

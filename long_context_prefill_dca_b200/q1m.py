@@ -66,10 +66,15 @@ SIGNATURES = {
                               PP, c_vp, c_vp, c_vp]),
     "q1m_attention_recall": (c_int, [c_vp, c_vp, c_i64, c_vp, c_vp]),
     "q1m_prefill_bounds": (c_i64, [c_i64, PP, c_vp, c_i64]),
+    "q1m_dca_sparse_prefill_chunks": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_int, c_int,
+                                              c_int, PP, c_i64, c_i64, c_vp, c_size, c_vp]),
     "q1m_dca_decode_scratch_bytes": (c_size, [c_int, c_int]),
     "q1m_dca_decode": (c_int, [c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_int, c_int, c_int, PP,
                                c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
     "q1m_status_poll": (c_int, [c_vp]),
+    "q1m_set_debug": (c_int, [c_int]),
+    "q1m_debug_enabled": (c_int, []),
+    "q1m_debug_inject": (c_int, [c_int]),
     "q1m_last_error": (ctypes.c_char_p, []),
     "q1m_version": (ctypes.c_char_p, []),
     "q1m_set_wait_budget": (c_int, [c_u64]),
@@ -150,6 +155,12 @@ def host_workspace_bytes(n, hq, hkv, d, p: Params) -> int:
 def dca_sparse_prefill(q, k, v, out, lse, n, hq, hkv, d, p: Params, ws, ws_bytes, stream=None):
     _call("q1m_dca_sparse_prefill", ptr(q), ptr(k), ptr(v), ptr(out), ptr(lse), n, hq, hkv, d,
           ctypes.byref(p), ptr(ws), ws_bytes, stream_handle(stream))
+
+
+def dca_sparse_prefill_chunks(q, k, v, out, lse, n, hq, hkv, d, p: Params, first, last, ws, ws_bytes,
+                              stream=None):
+    _call("q1m_dca_sparse_prefill_chunks", ptr(q), ptr(k), ptr(v), ptr(out), ptr(lse), n, hq, hkv,
+          d, ctypes.byref(p), int(first), int(last), ptr(ws), ws_bytes, stream_handle(stream))
 
 
 def dca_sparse_prefill_host(q, k, v, out, lse, n, hq, hkv, d, p: Params, ws, ws_bytes,
@@ -250,6 +261,23 @@ def prefill_bounds(w) -> list[tuple[int, int]]:
         out.append((s0, int(e)))
         s0 = int(e)
     return out
+
+
+def last_error() -> str:
+    """The calling thread's last error message from the library."""
+    return library().q1m_last_error().decode()
+
+
+def set_debug(on: bool) -> None:
+    _call("q1m_set_debug", 1 if on else 0)
+
+
+def debug_enabled() -> bool:
+    return bool(library().q1m_debug_enabled())
+
+
+def debug_inject(stage: str | int) -> None:
+    _call("q1m_debug_inject", STAGES.index(stage) if isinstance(stage, str) else int(stage))
 
 
 def status_poll(stream=None) -> int:

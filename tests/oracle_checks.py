@@ -460,3 +460,26 @@ def check_decode_row() -> float:
     ones = O.Oracle(q, k, np.ones_like(v), cfg)
     err = max(err, float(np.max(np.abs(ones.decode_row(cfg.seq_len - 1, 1)[0] - 1.0))))
     return err
+
+
+def check_key_order_invariance() -> float:
+    """The output does not depend on the order in which the attended keys are summed: the
+    oracle's rows against the same softmax taken over a random permutation of the (logit,
+    value) pairs of each row."""
+    cfg = tiny(yarn_s=2.0, vs_vertical=6, vs_slash=10, vs_force_local=4)
+    q, k, v = rand_qkv(cfg, 12)
+    orc = O.Oracle(q, k, v, cfg)
+    sel = orc.select_chunk(0, cfg.seq_len)
+    rows = np.array([5, 30, 61, 95])
+    got, _ = orc.attend_rows(rows, 0, sel)
+    rng = np.random.default_rng(3)
+    err = 0.0
+    for r, i in enumerate(rows):
+        js = np.nonzero(orc.attended(int(i), 0, sel))[0]
+        perm = rng.permutation(len(js))
+        jp = js[perm]
+        l = O.dca_logits(q[[i], 0, :], np.array([i]), orc.krot(0)[jp], jp, cfg)[0]
+        w = np.exp(l - l.max())
+        ref = (w[:, None] * v[jp, 0, :]).sum(0) / w.sum()
+        err = max(err, float(np.max(np.abs(got[r] - ref))))
+    return err

@@ -96,3 +96,34 @@ def test_decode_validates_before_launch():
     assert lib.q1m_dca_decode(*args(10, 1024, 4, 2, 128, nb - 1)) == -3        # scratch too small
     assert lib.q1m_dca_decode(None, 1, 1, 10, 256, 256, 1024, 4, 2, 128, ctypes.byref(p), 256, 256,
                               None, 256, nb, None) == -1                       # NULL pointer
+
+
+def test_chunk_range_validated():
+    import ctypes
+    from long_context_prefill_dca_b200 import q1m
+    from synth import configs as C
+    lib = q1m.library()
+    w = C.SMALL_SPARSE
+    p = q1m.params(w)
+    args = (1, 1, 1, 1, None, w.seq_len, w.n_q_heads, w.n_kv_heads, w.head_dim, ctypes.byref(p))
+    assert lib.q1m_dca_sparse_prefill_chunks(*args, -1, 2, 256, 1 << 40, None) == -1
+    assert lib.q1m_dca_sparse_prefill_chunks(*args, 3, 2, 256, 1 << 40, None) == -1
+
+
+def test_debug_mode_adds_guards_to_the_workspace():
+    from long_context_prefill_dca_b200 import q1m
+    from synth import configs as C
+    w = C.SMALL_SPARSE
+    args = (w.seq_len, w.n_q_heads, w.n_kv_heads, w.head_dim, q1m.params(w))
+    base = q1m.workspace_bytes(*args)
+    q1m.set_debug(True)
+    try:
+        assert q1m.debug_enabled()
+        dbg = q1m.workspace_bytes(*args)
+        assert dbg - base == 15 * 4096          # one guard after each of the 15 sparse-mode buffers
+    finally:
+        q1m.set_debug(False)
+    assert q1m.workspace_bytes(*args) == base and not q1m.debug_enabled()
+    with pytest.raises(q1m.Q1MError):
+        q1m.debug_inject(99)
+    q1m.debug_inject(-1)

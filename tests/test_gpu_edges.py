@@ -103,3 +103,24 @@ def test_nan_score_is_reported():
     q1m.vs_select(vert, slash, 300, 300, w.n_q_heads, q1m.params(w), V, S)
     assert q1m.status_poll() == -6
     assert q1m.status_poll() == 0
+
+
+def test_prefill_resumed_at_chunk_granularity():
+    """Chunks [0, 2) then [2, end) on the same workspace equal one call, bit for bit."""
+    w = BASE.with_(seq_len=1111, prefill_chunk=256)
+    x = I.generate(w)
+    g = {k: t.cuda() for k, t in x.items()}
+    layer = Layer(w)
+    whole = layer(g["q"], g["k"], g["v"]).clone()
+    lse_whole = torch.empty(w.n_q_heads, w.seq_len, device="cuda")
+    layer(g["q"], g["k"], g["v"], lse=lse_whole)
+    out = torch.full_like(whole, float("nan"))
+    lse = torch.full_like(lse_whole, float("nan"))
+    layer2 = Layer(w)
+    layer2.chunks(g["q"], g["k"], g["v"], 0, 2, out, lse)
+    torch.cuda.synchronize()
+    assert torch.isnan(out[512:]).all() and not torch.isnan(out[:512]).any()
+    layer2.chunks(g["q"], g["k"], g["v"], 2, 1 << 40, out, lse)
+    torch.cuda.synchronize()
+    q1m.check_status()
+    assert torch.equal(out, whole) and torch.equal(lse, lse_whole)

@@ -84,3 +84,7 @@ def test_equal_cost_chunks_fixture_and_invariants():
 
 def test_decode_row_brute_force():
     assert C.check_decode_row() < 1e-10
+
+
+def test_key_order_invariance():
+    assert C.check_key_order_invariance() < 1e-12
