@@ -114,8 +114,9 @@ q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, v
  * in the workspace, so chunks before first_chunk must have run on the same workspace (same
  * shapes and params) with nothing else written to it in between; the rows of out and lse
  * of the chunks that run are written, the others are left as they are. Running [0, a) and
- * then [a, end) gives the same result, bit for bit, as one q1m_dca_sparse_prefill call
- * (which is this call with [0, end)). */
+ * then [a, end) gives the same result as one q1m_dca_sparse_prefill call (which is this
+ * call with [0, end)): bit for bit in deterministic mode (q1m_set_deterministic), up to the
+ * rounding differences of the aligned tile order otherwise. */
 q1m_status q1m_dca_sparse_prefill_chunks(const void* q, const void* k, const void* v, void* out,
                                          float* lse, int64_t seq_len, int n_q_heads,
                                          int n_kv_heads, int head_dim, const q1m_params* p,
@@ -312,6 +313,22 @@ q1m_status q1m_dca_decode(const void* q, const void* k, const void* v, int64_t p
                           int n_kv_heads, int head_dim, const q1m_params* p, const float* table,
                           void* out, float* lse, void* scratch, size_t scratch_bytes,
                           void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Determinism
+ * ------------------------------------------------------------------------------------- */
+
+/* By default the attention kernel starts each work item's walk over its key blocks at a
+ * position taken from a global count of the tiles all CTAs have issued, so that CTAs
+ * streaming the same K/V range stay at about the same tile and share it in L2 (less DRAM
+ * traffic, and under the power cap a higher clock). The result does not depend on the tile
+ * order beyond rounding (fp32 sums and the fp16 rounding of P against the running maximum),
+ * but the order then depends on timing, so repeated runs can differ at that level (about
+ * 1e-4 relative). Deterministic mode (process-wide; initially on when the
+ * environment variable Q1M_DETERMINISTIC is set to a non-zero value) starts every walk at
+ * its first block: repeated runs, and the layer against its stages, are then bit-identical. */
+q1m_status q1m_set_deterministic(int on);
+int q1m_deterministic(void);
 
 /* ---------------------------------------------------------------------------------------
  * Debug mode

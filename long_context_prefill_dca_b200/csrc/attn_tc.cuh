@@ -65,6 +65,7 @@ struct K3Args {
   float* lse_part;       // [3][hq][ld_rows]
   const int32_t* units;  // sorted (pair << 2 | pattern)
   const int32_t* n_units;
+  int aligned;           // 1: walks start at the global cursor; 0: at lo (deterministic order)
 };
 
 struct K3Item {
@@ -137,8 +138,22 @@ struct K3Smem {
   uint64_t k_full[K3_NK], k_empty[K3_NK], v_full[K3_NV], v_empty[K3_NV];
   uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_done[2], pv_done[2];
   uint64_t drain;
+  int walk_start[2];        // first key block of each item's walk (K loader -> V loader)
+  uint64_t start_full[2], start_empty[2];
   uint32_t tmem_base;
 };
+
+// Free-running count of the K tiles all CTAs have issued. An item's walk over its key blocks
+// starts at the block this count divided by the number of CTAs points to (wrapping around
+// its range): every CTA's position then follows the same global clock, so CTAs that stream
+// the same K/V range read about the same tile at the same time and it is fetched from DRAM
+// about once and served from L2 after that. Measured on B200 at 7B@1M under the power cap:
+// 8-12% faster per prefill chunk, the DRAM power saved going to the SM clock. The online
+// softmax is exact in any tile order up to rounding, but the rounding (fp32 sums, and P in
+// fp16 against the running maximum) follows the order, which now depends on timing: runs can
+// differ at that level (about 1e-4 relative). With `aligned` off every walk starts at lo and
+// runs are bit-identical.
+__device__ unsigned long long g_k3_cursor;
 
 // --------------------------------------------------------------------------------------
 // Loader warps. Two warps walk the same tile sequence: ROLE 0 loads the Q views and the K
@@ -176,6 +191,7 @@ __device__ void k3_producer(K3Smem<D>& sm, const K3Args& a, const CUtensorMap* m
   const uint16_t* src = ROLE == 0 ? a.k_rot : a.v16;
   const bool leader = lane_id() == 0;
   uint32_t kt = 0;             // tiles produced by this CTA
+  uint32_t wn = 0;             // key-block walks started (items with key blocks)
   uint32_t qn[2] = {0, 0};     // Q loads per slot
   bool ok = true;
   auto stage_buf = [&](int st) -> uint8_t* { return ROLE == 0 ? sm.k[st] : sm.v[st]; };
@@ -216,38 +232,70 @@ __device__ void k3_producer(K3Smem<D>& sm, const K3Args& a, const CUtensorMap* m
         ++kt;
       }
     }
-    // key blocks: union of both slots' lists
+    // key blocks: union of both slots' lists, walked from a start block taken from the
+    // global tile count (the K loader picks it and hands it to the V loader) and wrapping
     int lo = 1 << 30, hi = -1;
 #pragma unroll
     for (int s = 0; s < 2; ++s)
       if (I.ntiles[s] > 0 && I.hi[s] >= I.lo[s]) { lo = min(lo, I.lo[s]); hi = max(hi, I.hi[s]); }
-    for (int w = lo >> 5; w <= (hi >> 5) && hi >= 0 && ok; ++w) {
-      uint32_t m0 = (I.ntiles[0] > 0) ? range_bits(w, I.lo[0], I.hi[0]) : 0u;
-      uint32_t m1 = (I.ntiles[1] > 0) ? range_bits(w, I.lo[1], I.hi[1]) : 0u;
-      if (a.mask) {
-        if (m0) m0 &= a.mask[((int64_t)I.h * a.nqb + I.qb[0]) * a.nkw + w];
-        if (m1) m1 &= a.mask[((int64_t)I.h * a.nqb + I.qb[1]) * a.nkw + w];
-      }
-      uint32_t u = m0 | m1;
-      while (u && ok) {
-        const int b = __ffs(u) - 1;
-        u &= u - 1;
-        const int kb = 32 * w + b;
-        const int st = kt % NS;
-        ok = mbar_wait_warp(&empty[st], ((kt / NS) & 1) ^ 1);
-        if (!ok) break;
-        const int y = (int)((int64_t)I.g * a.ld_tokens + (int64_t)kb * 128);
-        if (leader) {
-          if (ROLE == 0) {
-            sm.desc[st][0] = (int)((m0 >> b) & 1u) | (int)(((m1 >> b) & 1u) << 1);
-            sm.desc[st][1] = (int)(kb == I.B[0]) | ((int)(kb == I.B[1]) << 1);
-            sm.desc[st][2] = 128;
-          }
-          mbar_expect_tx(&full[st], TILE);
-#pragma unroll
-          for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(stage_buf(st) + hf * 16384, map, &full[st], 64 * hf, y);
+    auto walk = [&](int a0, int b0) {
+      for (int w = a0 >> 5; w <= (b0 >> 5) && b0 >= a0 && ok; ++w) {
+        uint32_t m0 = (I.ntiles[0] > 0) ? range_bits(w, max(I.lo[0], a0), min(I.hi[0], b0)) : 0u;
+        uint32_t m1 = (I.ntiles[1] > 0) ? range_bits(w, max(I.lo[1], a0), min(I.hi[1], b0)) : 0u;
+        if (a.mask) {
+          if (m0) m0 &= a.mask[((int64_t)I.h * a.nqb + I.qb[0]) * a.nkw + w];
+          if (m1) m1 &= a.mask[((int64_t)I.h * a.nqb + I.qb[1]) * a.nkw + w];
         }
-        ++kt;
+        uint32_t u = m0 | m1;
+        while (u && ok) {
+          const int b = __ffs(u) - 1;
+          u &= u - 1;
+          const int kb = 32 * w + b;
+          const int st = kt % NS;
+          ok = mbar_wait_warp(&empty[st], ((kt / NS) & 1) ^ 1);
+          if (!ok) break;
+          const int y = (int)((int64_t)I.g * a.ld_tokens + (int64_t)kb * 128);
+          if (leader) {
+            if (ROLE == 0) {
+              sm.desc[st][0] = (int)((m0 >> b) & 1u) | (int)(((m1 >> b) & 1u) << 1);
+              sm.desc[st][1] = (int)(kb == I.B[0]) | ((int)(kb == I.B[1]) << 1);
+              sm.desc[st][2] = 128;
+            }
+            mbar_expect_tx(&full[st], TILE);
+#pragma unroll
+            for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(stage_buf(st) + hf * 16384, map, &full[st], 64 * hf, y);
+            if (ROLE == 0 && a.aligned) atomicAdd(&g_k3_cursor, 1ull);
+          }
+          ++kt;
+        }
+      }
+    };
+    if (ok && hi >= lo) {
+      const int slot = (int)(wn & 1u);
+      int start = lo;
+      if (ROLE == 0) {
+        ok = mbar_wait_warp(&sm.start_empty[slot], ((wn >> 1) & 1u) ^ 1u);
+        if (ok && a.aligned) {
+          unsigned long long c = 0;
+          if (leader) c = *(volatile unsigned long long*)&g_k3_cursor;
+          c = __shfl_sync(0xFFFFFFFFu, c, 0);
+          start = lo + (int)((c / gridDim.x) % (unsigned long long)(hi - lo + 1));
+        }
+        if (ok) {
+          if (leader) { sm.walk_start[slot] = start; mbar_arrive(&sm.start_full[slot]); }
+        }
+      } else {
+        ok = mbar_wait_warp(&sm.start_full[slot], (wn >> 1) & 1u);
+        if (ok) {
+          start = sm.walk_start[slot];
+          __syncwarp();
+          if (leader) mbar_arrive(&sm.start_empty[slot]);
+        }
+      }
+      ++wn;
+      if (ok) {
+        walk(start, hi);
+        walk(lo, start - 1);
       }
     }
   }
@@ -549,6 +597,7 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap mq, const __grid_co
       mbar_init(&sm.pv_done[s], 1);
     }
     mbar_init(&sm.drain, 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&sm.start_full[i], 1); mbar_init(&sm.start_empty[i], 1); }
     fence_mbar_init();
   }
   if (w == 9) { tmem_alloc(&sm.tmem_base, 512); tmem_relinquish(); }

@@ -241,6 +241,17 @@ constexpr size_t GUARD_BYTES = 4096;
 constexpr uint32_t GUARD_WORD = 0xA5A5A5A5u;
 constexpr int MAX_GUARDS = 32;
 std::atomic<int> g_debug{-1};
+std::atomic<int> g_determ{-1};
+
+bool deterministic_on() {
+  int v = g_determ.load();
+  if (v < 0) {
+    const char* e = std::getenv("Q1M_DETERMINISTIC");
+    v = (e && *e && std::strcmp(e, "0") != 0) ? 1 : 0;
+    g_determ.store(v);
+  }
+  return v == 1;
+}
 std::atomic<int> g_inject{-1};
 
 bool debug_on() {
@@ -495,6 +506,7 @@ q1m_status run_attn_d(const uint16_t* qv, int64_t ld_rows, const uint16_t* k_rot
   a.o_part = o_part; a.lse_part = lse_part;
   a.units = units + 8;
   a.n_units = units;
+  a.aligned = deterministic_on() ? 0 : 1;
   const int U = 3 * a.npair;
   k3_units_kernel<<<1, 1024, (size_t)U * 4, st>>>(s0, a.nqb, a.L, units + 8, units);
   Q1M_LAUNCHED();
@@ -923,6 +935,13 @@ q1m_status q1m_status_poll(void* stream) {
   }
   return Q1M_OK;
 }
+
+q1m_status q1m_set_deterministic(int on) {
+  g_determ.store(on ? 1 : 0);
+  return Q1M_OK;
+}
+
+int q1m_deterministic(void) { return deterministic_on() ? 1 : 0; }
 
 q1m_status q1m_set_debug(int on) {
   g_debug.store(on ? 1 : 0);

@@ -72,6 +72,8 @@ SIGNATURES = {
     "q1m_dca_decode": (c_int, [c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_int, c_int, c_int, PP,
                                c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
     "q1m_status_poll": (c_int, [c_vp]),
+    "q1m_set_deterministic": (c_int, [c_int]),
+    "q1m_deterministic": (c_int, []),
     "q1m_set_debug": (c_int, [c_int]),
     "q1m_debug_enabled": (c_int, []),
     "q1m_debug_inject": (c_int, [c_int]),
@@ -266,6 +268,14 @@ def prefill_bounds(w) -> list[tuple[int, int]]:
 def last_error() -> str:
     """The calling thread's last error message from the library."""
     return library().q1m_last_error().decode()
+
+
+def set_deterministic(on: bool) -> None:
+    _call("q1m_set_deterministic", 1 if on else 0)
+
+
+def deterministic() -> bool:
+    return bool(library().q1m_deterministic())
 
 
 def set_debug(on: bool) -> None:

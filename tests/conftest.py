@@ -18,3 +18,16 @@ def cuda_lib():
     """The C-ABI library through its Python binding; fails loudly when absent."""
     from long_context_prefill_dca_b200 import q1m
     return q1m.library()
+
+
+@pytest.fixture
+def deterministic():
+    """Deterministic mode for a test that compares two runs bit for bit (the attention
+    kernel then walks every item's key blocks in a fixed order)."""
+    from long_context_prefill_dca_b200 import q1m
+    was = q1m.deterministic()
+    q1m.set_deterministic(True)
+    try:
+        yield
+    finally:
+        q1m.set_deterministic(was)

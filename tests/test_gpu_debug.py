@@ -24,7 +24,7 @@ def debug():
 
 @pytest.mark.parametrize("w", [C.SMALL_SPARSE, C.SMALL_DENSE_D128, C.SMALL_SPARSE.with_(equal_cost_chunks=3)],
                          ids=["sparse", "dense", "equal-cost"])
-def test_debug_mode_results_unchanged(w, debug):
+def test_debug_mode_results_unchanged(w, debug, deterministic):
     x = I.generate(w)
     g = {k: t.cuda() for k, t in x.items()}
     got = Layer(w)(g["q"], g["k"], g["v"])
