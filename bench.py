@@ -37,11 +37,23 @@ KERNEL_SOURCES = ("attn_tc.cuh", "q1m_device.cuh", "exp2_poly.h")
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "block_sparse_attn_dram_7b-1m.md")
 
 
+def kernel_source_hash() -> str:
+    """sha256 of the attention kernel's sources with comments and blank space removed, so
+    that it follows code changes only."""
+    import hashlib
+    import re
+    csrc = os.path.join(ROOT, "long_context_prefill_dca_b200", "csrc")
+    text = "".join(open(os.path.join(csrc, f)).read() for f in KERNEL_SOURCES)
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    text = re.sub(r"\s+", " ", text).strip()
+    return hashlib.sha256(text.encode()).hexdigest()
+
+
 def kernel_traffic(workload: str):
     """DRAM bytes per attention launch from the committed ncu summary of the 7B@1M layer, or
-    None when the workload differs or the kernel's sources changed since the capture (their
-    sha256 is recorded beside the figure)."""
-    import hashlib
+    None when the workload differs or the kernel's code changed since the capture (the hash
+    of its sources is recorded beside the figure)."""
     if workload != "7b-1m" or not os.path.exists(TRAFFIC_PROFILE):
         return None
     rec = {}
@@ -49,9 +61,7 @@ def kernel_traffic(workload: str):
         if ":" in line and line.split(":", 1)[0] in ("traffic_per_launch_bytes", "kernel_source_sha256"):
             k, v = line.split(":", 1)
             rec[k] = v.strip()
-    csrc = os.path.join(ROOT, "long_context_prefill_dca_b200", "csrc")
-    h = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read() for f in KERNEL_SOURCES)).hexdigest()
-    if rec.get("kernel_source_sha256") != h or "traffic_per_launch_bytes" not in rec:
+    if rec.get("kernel_source_sha256") != kernel_source_hash() or "traffic_per_launch_bytes" not in rec:
         return None
     return float(rec["traffic_per_launch_bytes"])
 

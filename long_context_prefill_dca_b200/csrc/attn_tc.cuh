@@ -14,10 +14,14 @@
 //    their key-block lists, each tile flagged with the slots that use it. Slot 1 is the
 //    block right after slot 0, so in dense mode the lists coincide and in sparse mode
 //    (Toeplitz block masks) they mostly do.
+//  * Each item walks its key blocks from a start taken from a global count of the tiles all
+//    CTAs have issued (wrapping around its range), so CTAs that stream the same K/V range
+//    stay at about the same tile and share it in L2 (see g_k3_cursor); deterministic mode
+//    starts every walk at its first block.
 //  * Warp roles: warps 0-3 softmax of slot 0, warps 4-7 softmax of slot 1, warp 8 loads
 //    (TMA for key blocks, cp.async gathers for residual vertical columns), warp 9 issues
-//    tcgen05.mma and owns tensor memory, warp 10 loads V tiles, warp 11 idles; the softmax warpgroups take
-//    registers from the third warpgroup (setmaxnreg) to hold a whole S row.
+//    tcgen05.mma and owns tensor memory, warp 10 loads V tiles, warp 11 idles; the softmax
+//    warpgroups take registers from the third warpgroup (setmaxnreg) to hold a whole S row.
 //  * Tensor memory per slot: S (128 fp32 columns), O (D fp32 columns); the softmax writes
 //    P as packed fp16 over the first 64 columns of S and the PV product reads it from
 //    tensor memory (A operand), with V as an MN-major shared-memory operand.

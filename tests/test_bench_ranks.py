@@ -91,10 +91,6 @@ def test_kernel_traffic_tracks_the_capture(tmp_path, monkeypatch):
     fake.write_text("traffic_per_launch_bytes: 123\nkernel_source_sha256: 00\n")
     monkeypatch.setattr(bench, "TRAFFIC_PROFILE", str(fake))
     assert bench.kernel_traffic("7b-1m") is None
-    import hashlib
-    import os
-    csrc = os.path.join(bench.ROOT, "long_context_prefill_dca_b200", "csrc")
-    h = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read()
-                                for f in bench.KERNEL_SOURCES)).hexdigest()
+    h = bench.kernel_source_hash()
     fake.write_text(f"traffic_per_launch_bytes: 123\nkernel_source_sha256: {h}\n")
     assert bench.kernel_traffic("7b-1m") == 123.0
