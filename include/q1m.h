@@ -22,8 +22,8 @@
  *     q1m_status is returned (q1m_last_error() gives a message). Otherwise the work is
  *     queued on `stream` (a cudaStream_t, NULL = legacy default stream) and the call returns
  *     Q1M_OK at once. Device-side faults detected by the kernels (a bounded wait that ran
- *     out, an fp16 range overflow, a NaN score) are latched on the device and returned by
- *     q1m_status_poll().
+ *     out, an fp16 range overflow, a NaN score, and in debug mode an overwritten guard region
+ *     or a malformed index list) are latched on the device and returned by q1m_status_poll().
  *   - Calls are thread-safe as long as concurrent calls use distinct workspaces/outputs.
  *   - head_dim is 64 or 128; n_q_heads is a multiple of n_kv_heads; (dca_chunk - local_window)
  *     and prefill_chunk are multiples of 128. Only sm_100a devices are supported; there is no
@@ -95,8 +95,8 @@ int64_t q1m_prefill_bounds(int64_t seq_len, const q1m_params* p, int64_t* ends, 
 size_t q1m_workspace_bytes(int64_t seq_len, int n_q_heads, int n_kv_heads, int head_dim,
                            const q1m_params* p);
 
-/* The layer: for every prefill chunk [s0, e) (s0 = p * prefill_chunk, e = min(N, s0 + P)),
- * rotate the chunk's keys and queries (DCA views), estimate vertical/slash scores from the
+/* The layer: for every prefill chunk [s0, e) (the bounds q1m_prefill_bounds lists: fixed
+ * chunks of prefill_chunk rows, or equal-cost chunks when equal_cost_chunks > 0), rotate the chunk's keys and queries (DCA views), estimate vertical/slash scores from the
  * chunk's last vs_last_q rows over keys [0, e), select the per-head budgets, build the
  * 128 x 128 block mask, run block-sparse DCA attention for rows [s0, e) and merge the three
  * DCA patterns' partial results ([P2] 四; [P5] Sparse Attention).
@@ -216,7 +216,9 @@ size_t q1m_attn_scratch_bytes(int64_t s0, int64_t e, int n_q_heads, int head_dim
  *   o_part[x][h][i - s0][:] = softmax-weighted sum of v (fp32), lse_part[x][h][i - s0] =
  *   log2-sum-exp2 of the log2-scaled logits (-inf when the segment is empty for the row).
  * qv, k_rot, v16: stage outputs above; mask/resid/cnt: q1m_vs_build_masks output or NULL.
- * o_part: device fp32 [3][Hq][ld_rows][D]; lse_part: device fp32 [3][Hq][ld_rows]. */
+ * o_part: device fp32 [3][Hq][ld_rows][D]; lse_part: device fp32 [3][Hq][ld_rows].
+ * The order in which a work item visits its key blocks follows a global tile count unless
+ * deterministic mode is on (q1m_set_deterministic); results agree up to rounding either way. */
 q1m_status q1m_block_sparse_attn(const uint16_t* qv, int64_t ld_rows, const uint16_t* k_rot,
                                  const uint16_t* v16, int64_t ld_tokens, const uint32_t* mask,
                                  const int32_t* resid, const int32_t* cnt, int64_t s0,
@@ -275,8 +277,8 @@ q1m_status q1m_attention_recall(const float* lse_sparse, const float* lse_dense,
  * ------------------------------------------------------------------------------------- */
 
 /* Synchronizes `stream`, then returns and clears the device-side status latched by the
- * kernels on the current device (Q1M_OK, Q1M_ERR_TIMEOUT or Q1M_ERR_RANGE), or
- * Q1M_ERR_CUDA if the stream reported an error. */
+ * kernels on the current device (Q1M_OK, Q1M_ERR_TIMEOUT, Q1M_ERR_RANGE or, in debug mode,
+ * Q1M_ERR_CHECK), or Q1M_ERR_CUDA if the stream reported an error. */
 q1m_status q1m_status_poll(void* stream);
 
 /* The message of the last failing call on this thread ("" if none). */
