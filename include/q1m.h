@@ -128,10 +128,17 @@ q1m_status q1m_dca_sparse_prefill_chunks(const void* q, const void* k, const voi
 size_t q1m_host_workspace_bytes(int64_t seq_len, int n_q_heads, int n_kv_heads, int head_dim,
                                 const q1m_params* p);
 
-/* The same layer from host buffers: copies q/k/v host->device (cudaMemcpyAsync, one per
- * tensor), runs q1m_dca_sparse_prefill, copies out (and lse if non-null) back, then
- * synchronizes `stream`. Host buffers should be pinned for full copy bandwidth. Returns the
- * device-side status of the run. */
+/* The same layer from host buffers, with the copies overlapping the compute one prefill
+ * chunk at a time: chunk c's rows of q, k and v go host->device on a copy stream of the
+ * call's own while earlier chunks compute (chunk c reads only its own rows of them; earlier
+ * keys are in the workspace already rotated), and its rows of out (and of lse, if non-null)
+ * go device->host on a second copy stream while later chunks compute. One cudaMemcpyAsync
+ * per tensor and chunk (cudaMemcpy2DAsync for the [Hq][N] lse rows). The copies start after
+ * the work already queued on `stream`; the call creates its two copy streams and three
+ * events, makes `stream` wait for the last download, synchronizes `stream` and destroys them
+ * before it returns. Results are those of q1m_dca_sparse_prefill on the same inputs. Host
+ * buffers should be pinned (page-locked) for full copy bandwidth and for the overlap.
+ * Returns the device-side status of the run. */
 q1m_status q1m_dca_sparse_prefill_host(const void* q_host, const void* k_host,
                                        const void* v_host, void* out_host, float* lse_host,
                                        int64_t seq_len, int n_q_heads, int n_kv_heads,

@@ -752,11 +752,31 @@ q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, v
                                        ws_bytes, stream);
 }
 
+// Host-side hooks around each prefill chunk of prefill_range, called when the chunk's work
+// is enqueued (before its first stage and after its merge).
+struct ChunkHooks {
+  virtual q1m_status before(int64_t s0, int64_t e) = 0;
+  virtual q1m_status after(int64_t s0, int64_t e) = 0;
+};
+
+static q1m_status prefill_range(const void* q, const void* k, const void* v, void* out,
+                                float* lse, int64_t n, int hq, int hkv, int d,
+                                const q1m_params* p, int64_t first_chunk, int64_t last_chunk,
+                                void* ws, size_t ws_bytes, void* stream, ChunkHooks* hooks);
+
 q1m_status q1m_dca_sparse_prefill_chunks(const void* q, const void* k, const void* v, void* out,
                                          float* lse, int64_t n, int hq, int hkv, int d,
                                          const q1m_params* p, int64_t first_chunk,
                                          int64_t last_chunk, void* ws, size_t ws_bytes,
                                          void* stream) {
+  return prefill_range(q, k, v, out, lse, n, hq, hkv, d, p, first_chunk, last_chunk, ws, ws_bytes,
+                       stream, nullptr);
+}
+
+static q1m_status prefill_range(const void* q, const void* k, const void* v, void* out,
+                                float* lse, int64_t n, int hq, int hkv, int d,
+                                const q1m_params* p, int64_t first_chunk, int64_t last_chunk,
+                                void* ws, size_t ws_bytes, void* stream, ChunkHooks* hooks) {
   Q1M_TRY(check_shape(n, hq, hkv, d, p));
   if (first_chunk < 0 || last_chunk < first_chunk) return fail(Q1M_ERR_INVALID, "bad chunk range");
   if (!q || !k || !v || !out || !ws) return fail(Q1M_ERR_INVALID, "NULL pointer");
@@ -792,6 +812,7 @@ q1m_status q1m_dca_sparse_prefill_chunks(const void* q, const void* k, const voi
   for (int64_t ci = first_chunk; ci < (int64_t)ends.size() && ci < last_chunk; ++ci) {
     const int64_t s0 = ci == 0 ? 0 : ends[ci - 1], e = ends[ci];
     const bool first = ci == first_chunk;
+    if (hooks) Q1M_TRY(hooks->before(s0, e));
     pr = prof_begin(Q1M_STAGE_KEYS, st);
     Q1M_TRY(run_rope_keys(k, v, s0, e, hkv, d, p, table, k_rot, v16, L.ld_tokens, st));
     prof_end(pr, st);
@@ -839,9 +860,72 @@ q1m_status q1m_dca_sparse_prefill_chunks(const void* q, const void* k, const voi
     Q1M_TRY(run_merge(o_part, lse_part, 3, L.ld_rows, s0, e, n, hq, d, p->out_dtype, Ld, out, lse, st));
     prof_end(pr, st);
     Q1M_TRY(debug_after(L, ws, Q1M_STAGE_MERGE, first, st));
+    if (hooks) Q1M_TRY(hooks->after(s0, e));
   }
   return Q1M_OK;
 }
+
+// The host-buffer path's copies, one prefill chunk at a time on two copy streams of the
+// call's own: chunk c's rows of q, k and v go up on `up` while earlier chunks compute, and
+// its rows of out and lse come down on `down` while later chunks compute. A chunk reads
+// only its own rows of q, k and v (the rotated keys of earlier chunks are in the workspace),
+// so the compute stream waits only for that chunk's upload.
+struct HostCopies final : ChunkHooks {
+  const uint8_t *q_h = nullptr, *k_h = nullptr, *v_h = nullptr;
+  uint8_t* out_h = nullptr;
+  float* lse_h = nullptr;
+  uint8_t *dq = nullptr, *dk = nullptr, *dv = nullptr, *dout = nullptr;
+  float* dlse = nullptr;
+  size_t row_q = 0, row_k = 0, row_o = 0;   // bytes per token of q, of k (and v), of out
+  int64_t n = 0;
+  int hq = 0;
+  cudaStream_t st = nullptr, up = nullptr, down = nullptr;
+  cudaEvent_t ev_in = nullptr, ev_out = nullptr, ev_edge = nullptr;
+
+  q1m_status open() {
+    Q1M_CUDA(cudaStreamCreateWithFlags(&up, cudaStreamNonBlocking));
+    Q1M_CUDA(cudaStreamCreateWithFlags(&down, cudaStreamNonBlocking));
+    Q1M_CUDA(cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming));
+    Q1M_CUDA(cudaEventCreateWithFlags(&ev_out, cudaEventDisableTiming));
+    Q1M_CUDA(cudaEventCreateWithFlags(&ev_edge, cudaEventDisableTiming));
+    // the uploads start after the work already queued on the caller's stream
+    Q1M_CUDA(cudaEventRecord(ev_edge, st));
+    Q1M_CUDA(cudaStreamWaitEvent(up, ev_edge, 0));
+    return Q1M_OK;
+  }
+  q1m_status before(int64_t s0, int64_t e) override {
+    const size_t r = (size_t)(e - s0);
+    Q1M_CUDA(cudaMemcpyAsync(dq + s0 * row_q, q_h + s0 * row_q, r * row_q, cudaMemcpyHostToDevice, up));
+    Q1M_CUDA(cudaMemcpyAsync(dk + s0 * row_k, k_h + s0 * row_k, r * row_k, cudaMemcpyHostToDevice, up));
+    Q1M_CUDA(cudaMemcpyAsync(dv + s0 * row_k, v_h + s0 * row_k, r * row_k, cudaMemcpyHostToDevice, up));
+    Q1M_CUDA(cudaEventRecord(ev_in, up));
+    Q1M_CUDA(cudaStreamWaitEvent(st, ev_in, 0));
+    return Q1M_OK;
+  }
+  q1m_status after(int64_t s0, int64_t e) override {
+    const size_t r = (size_t)(e - s0);
+    Q1M_CUDA(cudaEventRecord(ev_out, st));
+    Q1M_CUDA(cudaStreamWaitEvent(down, ev_out, 0));
+    Q1M_CUDA(cudaMemcpyAsync(out_h + s0 * row_o, dout + s0 * row_o, r * row_o, cudaMemcpyDeviceToHost, down));
+    if (lse_h)   // rows [s0, e) of every head of the [Hq][N] array
+      Q1M_CUDA(cudaMemcpy2DAsync(lse_h + s0, (size_t)n * 4, dlse + s0, (size_t)n * 4, r * 4, hq,
+                                 cudaMemcpyDeviceToHost, down));
+    return Q1M_OK;
+  }
+  // the caller's stream then follows the downloads
+  q1m_status close() {
+    Q1M_CUDA(cudaEventRecord(ev_edge, down));
+    Q1M_CUDA(cudaStreamWaitEvent(st, ev_edge, 0));
+    return Q1M_OK;
+  }
+  ~HostCopies() {
+    if (up) { cudaStreamSynchronize(up); cudaStreamDestroy(up); }
+    if (down) { cudaStreamSynchronize(down); cudaStreamDestroy(down); }
+    if (ev_in) cudaEventDestroy(ev_in);
+    if (ev_out) cudaEventDestroy(ev_out);
+    if (ev_edge) cudaEventDestroy(ev_edge);
+  }
+};
 
 q1m_status q1m_dca_sparse_prefill_host(const void* q_h, const void* k_h, const void* v_h, void* out_h,
                                        float* lse_h, int64_t n, int hq, int hkv, int d,
@@ -858,14 +942,27 @@ q1m_status q1m_dca_sparse_prefill_host(const void* q_h, const void* k_h, const v
   void* dv = at<void>(ws, off); off += align_up(bk);
   void* dout = at<void>(ws, off); off += align_up(bo);
   float* dlse = at<float>(ws, off); off += align_up((size_t)n * hq * 4);
-  cudaStream_t st = S(stream);
-  Q1M_CUDA(cudaMemcpyAsync(dq, q_h, bq, cudaMemcpyHostToDevice, st));
-  Q1M_CUDA(cudaMemcpyAsync(dk, k_h, bk, cudaMemcpyHostToDevice, st));
-  Q1M_CUDA(cudaMemcpyAsync(dv, v_h, bk, cudaMemcpyHostToDevice, st));
-  Q1M_TRY(q1m_dca_sparse_prefill(dq, dk, dv, dout, lse_h ? dlse : nullptr, n, hq, hkv, d, p,
-                                 at<void>(ws, off), ws_bytes - off, stream));
-  Q1M_CUDA(cudaMemcpyAsync(out_h, dout, bo, cudaMemcpyDeviceToHost, st));
-  if (lse_h) Q1M_CUDA(cudaMemcpyAsync(lse_h, dlse, (size_t)n * hq * 4, cudaMemcpyDeviceToHost, st));
+  HostCopies hc;
+  hc.q_h = static_cast<const uint8_t*>(q_h);
+  hc.k_h = static_cast<const uint8_t*>(k_h);
+  hc.v_h = static_cast<const uint8_t*>(v_h);
+  hc.out_h = static_cast<uint8_t*>(out_h);
+  hc.lse_h = lse_h;
+  hc.dq = static_cast<uint8_t*>(dq);
+  hc.dk = static_cast<uint8_t*>(dk);
+  hc.dv = static_cast<uint8_t*>(dv);
+  hc.dout = static_cast<uint8_t*>(dout);
+  hc.dlse = dlse;
+  hc.row_q = (size_t)hq * d * ein;
+  hc.row_k = (size_t)hkv * d * ein;
+  hc.row_o = (size_t)hq * d * eout;
+  hc.n = n;
+  hc.hq = hq;
+  hc.st = S(stream);
+  Q1M_TRY(hc.open());
+  Q1M_TRY(prefill_range(dq, dk, dv, dout, lse_h ? dlse : nullptr, n, hq, hkv, d, p, 0, INT64_MAX,
+                        at<void>(ws, off), ws_bytes - off, stream, &hc));
+  Q1M_TRY(hc.close());
   return q1m_status_poll(stream);
 }
 

@@ -69,17 +69,35 @@ def test_edge_case_matches_oracle(w):
     assert np.abs(lse.cpu().numpy() - ref_lse).max() <= 2e-3
 
 
-def test_host_buffer_entry_point_matches_device_entry_point(deterministic):
-    w = BASE
+HOST_CASES = [BASE, BASE.with_(name="host-ragged-many", seq_len=1111, prefill_chunk=128),
+              BASE.with_(name="host-equal-cost", seq_len=1500, equal_cost_chunks=3),
+              BASE.with_(name="host-one-chunk", prefill_chunk=1024)]
+
+
+@pytest.mark.parametrize("w", HOST_CASES, ids=lambda w: w.name)
+def test_host_buffer_entry_point_matches_device_entry_point(deterministic, w):
+    """The host-buffer path uploads and downloads chunk by chunk on its own copy streams;
+    its out and lse equal the device path's bit for bit."""
     x = I.generate(w)
     g = {k: t.cuda() for k, t in x.items()}
-    dev = Layer(w)(g["q"], g["k"], g["v"]).cpu()
+    lse_d = torch.empty(w.n_q_heads, w.seq_len, device="cuda")
+    dev = Layer(w)(g["q"], g["k"], g["v"], lse=lse_d).cpu()
     pin = {k: v.pin_memory() for k, v in x.items()}
-    out_h = torch.empty(dev.shape, dtype=dev.dtype).pin_memory()
-    lse_h = torch.empty(w.n_q_heads, w.seq_len).pin_memory()
+    out_h = torch.full(dev.shape, float("nan"), dtype=dev.dtype).pin_memory()
+    lse_h = torch.full((w.n_q_heads, w.seq_len), float("nan")).pin_memory()
     HostLayer(w)(pin["q"], pin["k"], pin["v"], out_h, lse_h)
     assert torch.equal(out_h, dev)
-    assert torch.isfinite(lse_h).all()
+    assert torch.equal(lse_h, lse_d.cpu())
+    # a second call on a side stream, with other inputs queued on it first, gives the same
+    x2 = I.generate(w.with_(seed=w.seed + 1))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        junk = torch.empty(64 << 20, dtype=torch.uint8, device="cuda").fill_(7)   # queued work
+        HostLayer(w)(*(x2[k].pin_memory() for k in ("q", "k", "v")), out_h, lse_h,
+                     stream=s.cuda_stream)
+    ref2 = Layer(w)(*(x2[k].cuda() for k in ("q", "k", "v"))).cpu()
+    assert torch.equal(out_h, ref2)
+    del junk
 
 
 def test_fp16_range_overflow_is_reported():
