@@ -127,3 +127,35 @@ def test_debug_mode_adds_guards_to_the_workspace():
     with pytest.raises(q1m.Q1MError):
         q1m.debug_inject(99)
     q1m.debug_inject(-1)
+
+
+def test_c_consumer_compiles_as_c_and_links(lib, tmp_path):
+    """The header is valid C11 and the library links from C: a plain C program calls the
+    GPU-free entry points and prints what the Python binding also sees."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not found")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(build.LIB)
+    exe = str(tmp_path / "abi_consumer")
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(root, "include"), os.path.join(root, "tests", "abi_consumer.c"),
+                    "-L", libdir, "-l:" + os.path.basename(build.LIB), "-Wl,-rpath," + libdir,
+                    "-o", exe], check=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout.splitlines()
+    got = {line.split(" ", 1)[0]: line.split(" ", 1)[1] for line in out}
+    assert got["version"] == q1m.version()
+    w = C.Workload(name="c", seq_len=1500, n_q_heads=4, n_kv_heads=2, head_dim=128,
+                   in_dtype="bf16", rope_base=1e4, dca_chunk=384, local_window=128, yarn_s=2.0,
+                   prefill_chunk=256, vs_vertical=20, vs_slash=70, vs_last_q=64, vs_force_local=8)
+    for tag, ww in (("fixed", w), ("equal", w.with_(equal_cost_chunks=3))):
+        ends = [e for _, e in q1m.prefill_bounds(ww)]
+        assert got[tag].split() == [str(len(ends))] + [str(e) for e in ends], (tag, got[tag])
+    assert got["too_many"] == "-3"
+    p = q1m.params(w, "f32")
+    assert int(got["workspace"]) == lib.q1m_workspace_bytes(1500, 4, 2, 128, ctypes.byref(p)) > 0
+    assert int(got["host_workspace"]) == lib.q1m_host_workspace_bytes(1500, 4, 2, 128, ctypes.byref(p))
+    assert int(got["decode_scratch"]) == q1m.dca_decode_scratch_bytes(4, 128) > 0
+    assert got["null_status"] == "-1" and got["null_message"]
