@@ -4,7 +4,7 @@
 
 Builds the fp16 cache of the first n - 1 tokens with the prefill's key rotation, then times
 the decode step of the token at n - 1 (append, query views, decode kernel, merge) for a few
-context lengths. The decode kernel is HBM-bound: its algorithmic bytes are the K and V rows
+context lengths, called eagerly and replayed from a CUDA graph. The decode kernel is HBM-bound: its algorithmic bytes are the K and V rows
 it reads, 2 x (pos + 1) x Hkv x D x 2; the roofline is the measured copy bandwidth. The K/V
 read per step (2.1 GB at 1M) is far larger than L2, so no flush is needed. One JSON line per
 context length.
@@ -70,15 +70,39 @@ def main():
         prof = q1m.profile_read()
         q1m.profile_enable(False)
         step_us = e0.elapsed_time(e1) / args.steps * 1e3
+        # the same step replayed from a CUDA graph: the device-side step time without the
+        # host's per-call work (argument marshalling, four launches), which dominates at
+        # short contexts; a serving loop would capture the step the same way
+        gs = torch.cuda.Stream()
+        gs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(gs):
+            step()
+        torch.cuda.current_stream().wait_stream(gs)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+            step()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        q1m.check_status()
+        graph_us = e0.elapsed_time(e1) / args.steps * 1e3
+        del graph
         k_ms, k_n = prof["decode"]
         kern_us = k_ms / k_n * 1e3
         byts = 2.0 * (pos + 1) * w.n_kv_heads * w.head_dim * 2
         gbs = byts / (kern_us * 1e-6) / 1e9
         print(json.dumps({"workload": w.name, "context": pos + 1, "step_us": step_us,
-                          "decode_kernel_us": kern_us, "kv_bytes": byts,
+                          "step_graph_us": graph_us, "decode_kernel_us": kern_us,
+                          "kv_bytes": byts,
                           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                                        "frac": gbs / peak, "peak_source": src},
-                          "tokens_per_s_per_layer": 1e6 / step_us}), flush=True)
+                          "tokens_per_s_per_layer": 1e6 / step_us,
+                          "tokens_per_s_per_layer_graph": 1e6 / graph_us}), flush=True)
     # restore the cache row n - 1 is not needed: the cache is discarded
 
 
