@@ -385,24 +385,60 @@ def check_attended_set() -> bool:
     return bool(ok)
 
 
+def check_residual_verticals() -> bool:
+    """The residual vertical columns of a query block, together with its computed blocks,
+    give exactly the attended set of every row of the block (no selected column lost or
+    counted twice); they lie outside the computed blocks, ascend, and never pass the block's
+    last row."""
+    rng = np.random.default_rng(21)
+    bs = O.BLOCK
+    ok = True
+    for t in range(40):
+        e = int(rng.integers(1, 700))
+        b = int(rng.integers(0, (e - 1) // bs + 1))
+        r0, r1 = b * bs, min(b * bs + bs - 1, e - 1)
+        V = rng.choice(e, size=min(e, int(rng.integers(0, 40))), replace=False)
+        if t % 2:          # the block's own first and last rows among the columns
+            V = np.concatenate([V, [r0, r1]])
+        V = np.unique(V)
+        lo_o = bs if t % 4 >= 2 and e > bs else 0     # no short offsets: diagonal block may be skipped
+        S = np.sort(rng.choice(np.arange(lo_o, e), size=min(e - lo_o, int(rng.integers(1, 30))),
+                               replace=False))
+        blocks = O.computed_blocks(S, b, e)
+        res = np.asarray(O.residual_verticals(V, blocks, b, e))
+        ok &= bool(np.all(np.diff(res) > 0)) and bool(np.all(res <= r1))
+        ok &= not bool(np.any(blocks[res // bs])) if len(res) else True
+        for i in range(r0, r1 + 1):
+            parts = blocks[np.arange(i + 1) // bs].copy()
+            parts[res[res <= i]] = True
+            ok &= bool(np.array_equal(O.attended_mask(i, blocks, V), parts))
+    return bool(ok)
+
+
 def check_recall() -> float:
-    """Recall is 1 for a full budget and equals exp(lse_sparse - lse_dense) otherwise."""
-    cfg = tiny(seq_len=260, dca_chunk=80, local_window=16, vs_vertical=4, vs_slash=12,
-               vs_force_local=4, prefill_chunk=260)
-    q, k, v = rand_qkv(cfg, 16)
-    orc = O.Oracle(q, k, v, cfg)
-    sel = orc.select_chunk(0, cfg.seq_len)
-    rows = np.array([3, 70, 129, 200, 259])
-    rec = orc.recall_rows(rows, 1, sel)
-    _, lse_s = orc.attend_rows(rows, 1, sel)
-    dense = O.Oracle(q, k, v, cfg.with_(vs_vertical=0, vs_slash=0))
-    _, lse_d = dense.attend_rows(rows, 1, O.ChunkSelection(0, cfg.seq_len))
-    full = cfg.with_(vs_vertical=10**6, vs_slash=10**6)
-    of = O.Oracle(q, k, v, full)
-    sf = of.select_chunk(0, cfg.seq_len)
-    return max(float(np.max(np.abs(rec - np.exp(lse_s - lse_d)))),
-               float(np.max(np.abs(of.recall_rows(rows, 1, sf) - 1.0))),
-               float(max(0.0, np.max(rec) - 1.0)))
+    """Recall is 1 for a full budget and equals exp(lse_sparse - lse_dense) otherwise, on a
+    layer whose selection covers every block and on a sparser one where rows keep only part
+    of the dense mass (the check fails if that second case does not reach recall < 0.9)."""
+    err, low = 0.0, 1.0
+    for n, ns, rows in ((260, 12, [3, 70, 129, 200, 259]), (1400, 4, [3, 129, 700, 1100, 1399])):
+        cfg = tiny(seq_len=n, dca_chunk=80, local_window=16, vs_vertical=4, vs_slash=ns,
+                   vs_force_local=2, prefill_chunk=n)
+        rows = np.array(rows)
+        q, k, v = rand_qkv(cfg, 16)
+        orc = O.Oracle(q, k, v, cfg)
+        sel = orc.select_chunk(0, cfg.seq_len)
+        rec = orc.recall_rows(rows, 1, sel)
+        _, lse_s = orc.attend_rows(rows, 1, sel)
+        dense = O.Oracle(q, k, v, cfg.with_(vs_vertical=0, vs_slash=0))
+        _, lse_d = dense.attend_rows(rows, 1, O.ChunkSelection(0, cfg.seq_len))
+        full = cfg.with_(vs_vertical=10**6, vs_slash=10**6)
+        of = O.Oracle(q, k, v, full)
+        sf = of.select_chunk(0, cfg.seq_len)
+        err = max(err, float(np.max(np.abs(rec - np.exp(lse_s - lse_d)))),
+                  float(np.max(np.abs(of.recall_rows(rows, 1, sf) - 1.0))),
+                  float(max(0.0, np.max(rec) - 1.0)))
+        low = min(low, float(np.min(rec)))
+    return err if low < 0.9 else float("inf")
 
 
 def check_equal_cost_chunks() -> int:

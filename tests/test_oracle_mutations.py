@@ -31,6 +31,12 @@ def _all_checks():
     res["attended"] = C.check_attended_set()
     res["chunks"] = _passes(C.check_equal_cost_chunks)
     res["decode"] = C.check_decode_row() < 1e-10
+    res["rope_rel"] = C.check_rope_relative() < 1e-10
+    res["causal"] = C.check_causal() < 1e-12
+    res["lse_merge"] = C.check_lse_merge() < 1e-12
+    res["recall"] = C.check_recall() < 1e-12
+    res["key_order"] = C.check_key_order_invariance() < 1e-12
+    res["residual"] = C.check_residual_verticals()
     return res
 
 
@@ -167,6 +173,63 @@ def _attended_without_verticals(i, blocks, V, bs=O.BLOCK):
     return blocks[js // bs].copy()
 
 
+def _key_at_j(j, cfg):
+    return np.asarray(j)
+
+
+def _softmax_unnormalised(l):
+    m = np.max(l, axis=1, keepdims=True)
+    p = np.exp(l - m)
+    return p, (m + np.log(np.sum(p, axis=1, keepdims=True)))[:, 0]
+
+
+def _merge_unnormalised(outs, lses):
+    m = np.max(lses, axis=0)
+    w = np.exp(lses - m[None, :])
+    return np.sum(w[:, :, None] * outs, axis=0), m + np.log(np.sum(w, axis=0))
+
+
+def _estimate_not_causal(q_R, R, krot_g, e, cfg):
+    js = np.arange(e)
+    p, lse = O.softmax_rows(O.dca_logits(q_R, R, krot_g[:e], js, cfg))
+    slash = np.zeros(e, dtype=np.float64)
+    for r, i in enumerate(R):
+        slash[: i + 1] += p[r, i::-1]
+    return np.sum(p, axis=0).astype(np.float32), slash.astype(np.float32), lse
+
+
+def _residual_inside_blocks(V, blocks, b, e, bs=O.BLOCK):
+    V = np.asarray(V)
+    return V[V <= min(b * bs + bs - 1, e - 1)]
+
+
+def _residual_cut_early(V, blocks, b, e, bs=O.BLOCK):
+    r1 = min(b * bs + bs - 1, e - 1)
+    V = np.asarray(V)
+    return V[(V < r1) & ~blocks[np.minimum(V // bs, blocks.shape[0] - 1)]]
+
+
+def _decode_without_own_key(self, pos, h):
+    js = np.arange(max(pos, 1))
+    l = O.dca_logits(self.q_rows(np.array([pos]), h), np.array([pos]),
+                     self.krot(h // self.cfg.group)[: len(js)], js, self.cfg)
+    p, lse = O.softmax_rows(l)
+    return (p @ self.v[: len(js), h // self.cfg.group, :])[0], float(lse[0])
+
+
+def _recall_squared(self, rows, h, sel):
+    rows = np.asarray(rows)
+    imax = int(rows.max())
+    js = np.arange(imax + 1)
+    l = O.dca_logits(self.q_rows(rows, h), rows, self.krot(h // self.cfg.group)[: imax + 1],
+                     js, self.cfg)
+    res = np.zeros(len(rows))
+    for r, i in enumerate(rows):
+        p, _ = O.softmax_rows(l[[r], : i + 1])
+        res[r] = float(np.sum(p[0][self.attended(int(i), h, sel)])) ** 2
+    return res
+
+
 MUTATIONS = [
     ("rope sign flipped", "rope", _rope_sign),
     ("rope pairs interleaved", "rope", _rope_interleaved),
@@ -188,12 +251,24 @@ MUTATIONS = [
     ("chunk target rounded down", "equal_cost_chunks", _chunks_variant(lambda b: b + 1, ceil_target=False)),
     ("repeated chunk boundaries kept", "equal_cost_chunks",
      _chunks_variant(lambda b: b + 1, drop_repeats=False)),
+    ("keys rotated at j instead of j mod L", "dca_key_position", _key_at_j),
+    ("softmax weights not normalised", "softmax_rows", _softmax_unnormalised),
+    ("LSE merge weights not normalised", "lse_merge", _merge_unnormalised),
+    ("estimator softmax not causal", "estimate_head", _estimate_not_causal),
+    ("residual verticals keep columns inside computed blocks", "residual_verticals",
+     _residual_inside_blocks),
+    ("residual verticals stop one row early", "residual_verticals", _residual_cut_early),
+    ("decode step leaves out the token's own key", "Oracle.decode_row", _decode_without_own_key),
+    ("recall squared", "Oracle.recall_rows", _recall_squared),
 ]
 
 
 @pytest.mark.parametrize("name,attr,fn", MUTATIONS, ids=[m[0] for m in MUTATIONS])
 def test_mutation_is_caught(monkeypatch, name, attr, fn):
-    monkeypatch.setattr(O, attr, fn)
+    owner = O
+    for part in attr.split(".")[:-1]:
+        owner = getattr(owner, part)
+    monkeypatch.setattr(owner, attr.split(".")[-1], fn)
     res = _all_checks()
     failed = [k for k, ok in res.items() if not ok]
     assert failed, f"no pin caught the planted mistake: {name}"

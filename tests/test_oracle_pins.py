@@ -88,3 +88,7 @@ def test_decode_row_brute_force():
 
 def test_key_order_invariance():
     assert C.check_key_order_invariance() < 1e-12
+
+
+def test_residual_verticals_complete_the_attended_set():
+    assert C.check_residual_verticals()
