@@ -102,7 +102,10 @@ size_t q1m_workspace_bytes(int64_t seq_len, int n_q_heads, int n_kv_heads, int h
  * DCA patterns' partial results ([P2] 四; [P5] Sparse Attention).
  * q: [N][Hq][D], k, v: [N][Hkv][D] in p->in_dtype; out: [N][Hq][D] in p->out_dtype;
  * lse (nullable): [Hq][N] fp32, natural-log log-sum-exp of each row's scaled logits.
- * workspace: device memory of at least q1m_workspace_bytes(...) bytes, 256-byte aligned. */
+ * workspace: device memory of at least q1m_workspace_bytes(...) bytes, 256-byte aligned.
+ * The call only enqueues work on `stream` (no host synchronization, no allocation), so it may
+ * be captured into a CUDA graph and replayed, with the stage timers (q1m_profile_enable)
+ * off; the key-block order follows q1m_set_deterministic as it stood at capture. */
 q1m_status q1m_dca_sparse_prefill(const void* q, const void* k, const void* v, void* out,
                                   float* lse, int64_t seq_len, int n_q_heads, int n_kv_heads,
                                   int head_dim, const q1m_params* p, void* workspace,

@@ -167,3 +167,54 @@ def test_repeated_runs_default_and_deterministic():
     for u in (d, a):
         diff = (c - u).abs()
         assert diff.max().item() <= 2e-3 and diff.sum().item() <= 5e-4 * c.abs().sum().item()
+
+
+def test_host_path_bf16_out_without_lse_and_pageable_buffers(deterministic):
+    """bf16 output with lse left out, from pinned and from pageable host buffers."""
+    w = BASE.with_(seq_len=900)
+    x = I.generate(w)
+    g = {k: t.cuda() for k, t in x.items()}
+    dev = Layer(w, "bf16")(g["q"], g["k"], g["v"]).cpu()
+    for pinned in (True, False):
+        src = {k: (t.pin_memory() if pinned else t.clone()) for k, t in x.items()}
+        out_h = torch.zeros(dev.shape, dtype=torch.bfloat16)
+        if pinned:
+            out_h = out_h.pin_memory()
+        HostLayer(w, "bf16")(src["q"], src["k"], src["v"], out_h, None)
+        assert torch.equal(out_h, dev), pinned
+
+
+def test_layer_replays_from_a_cuda_graph(deterministic):
+    """The whole layer (every prefill chunk's stages) captured into one CUDA graph: a replay
+    equals an eager call bit for bit, and new inputs copied into the captured buffers give
+    the new result."""
+    w = BASE.with_(seq_len=1111, prefill_chunk=256)
+    x = I.generate(w)
+    g = {k: t.cuda() for k, t in x.items()}
+    layer = Layer(w)
+    eager = layer(g["q"], g["k"], g["v"]).clone()
+    out = torch.empty_like(eager)
+    lse = torch.empty(w.n_q_heads, w.seq_len, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        layer(g["q"], g["k"], g["v"], out=out, lse=lse)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+        layer(g["q"], g["k"], g["v"], out=out, lse=lse)
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    q1m.check_status()
+    assert torch.equal(out, eager)
+    x2 = I.generate(w.with_(seed=w.seed + 7))
+    for k in ("q", "k", "v"):
+        g[k].copy_(x2[k].cuda())
+    graph.replay()
+    torch.cuda.synchronize()
+    q1m.check_status()
+    ref2 = Layer(w)(g["q"], g["k"], g["v"])
+    assert torch.equal(out, ref2)
+    del graph
