@@ -43,7 +43,8 @@ constexpr int K3_REGS_SOFTMAX = 192;
 constexpr int K3_REGS_OTHER = 120;
 constexpr float K3_RESCALE_THRESHOLD = 8.0f;
 // exponentials of K3_POLY_PAIRS_OF_8 of every 8 pairs run on the FMA pipe (ex2_poly2), the
-// rest on the MUFU; measured on B200 the softmax is not MUFU-bound, so the default is 0
+// rest on the MUFU; measured on B200 with both slots' softmax warps active, 2 to 4 of 8 on the
+// FMA pipe made the kernel 10-35% slower, so the default is 0
 constexpr int K3_POLY_PAIRS_OF_8 = 0;
 // P overwrites the first half of S, so the slot's next QK^T (which writes S) must not
 // overtake the PV MMA that reads P. tcgen05.mma operations issued by one thread execute in
