@@ -1,6 +1,7 @@
 /* A plain C11 consumer of the library's C ABI: it includes the header as C (not C++), links
  * the shared library and calls the entry points that need no GPU, printing one line each.
  * test_abi.py builds it with gcc, runs it and checks the lines against the Python binding. */
+#include <stddef.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -43,5 +44,22 @@ int main(void) {
                                          0, NULL);
   printf("null_status %d\n", (int)st);
   printf("null_message %s\n", q1m_last_error());
+
+  /* the parameter block's layout as the C compiler lays it out */
+#define FIELD(f) printf("offset_%s %zu\n", #f, offsetof(q1m_params, f))
+  printf("sizeof_params %zu\n", sizeof(q1m_params));
+  FIELD(in_dtype);
+  FIELD(out_dtype);
+  FIELD(rope_base);
+  FIELD(yarn_s);
+  FIELD(dca_chunk);
+  FIELD(local_window);
+  FIELD(vs_vertical);
+  FIELD(vs_slash);
+  FIELD(vs_last_q);
+  FIELD(vs_force_local);
+  FIELD(prefill_chunk);
+  FIELD(equal_cost_chunks);
+#undef FIELD
   return 0;
 }

@@ -159,3 +159,9 @@ def test_c_consumer_compiles_as_c_and_links(lib, tmp_path):
     assert int(got["host_workspace"]) == lib.q1m_host_workspace_bytes(1500, 4, 2, 128, ctypes.byref(p))
     assert int(got["decode_scratch"]) == q1m.dca_decode_scratch_bytes(4, 128) > 0
     assert got["null_status"] == "-1" and got["null_message"]
+    # the binding's parameter block has the C layout, field by field
+    assert int(got["sizeof_params"]) == ctypes.sizeof(q1m.Params)
+    for name, _ in q1m.Params._fields_:
+        assert int(got["offset_" + name]) == getattr(q1m.Params, name).offset, name
+    assert {k[len("offset_"):] for k in got if k.startswith("offset_")} == \
+        {n for n, _ in q1m.Params._fields_}
