@@ -165,3 +165,40 @@ def test_c_consumer_compiles_as_c_and_links(lib, tmp_path):
         assert int(got["offset_" + name]) == getattr(q1m.Params, name).offset, name
     assert {k[len("offset_"):] for k in got if k.startswith("offset_")} == \
         {n for n, _ in q1m.Params._fields_}
+
+
+def _c_kind(decl: str) -> str:
+    decl = decl.strip()
+    if "*" in decl:
+        return "ptr"
+    base = decl.replace("const ", "").split()[0]
+    return {"int": "i32", "int32_t": "i32", "q1m_status": "i32", "int64_t": "i64",
+            "uint64_t": "u64", "size_t": "u64", "double": "f64", "void": "void"}[base]
+
+
+def _ctypes_kind(t) -> str:
+    if t is None:
+        return "void"
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(t, "_type_") and t.__name__.startswith("LP_"):
+        return "ptr"
+    # size_t and uint64_t are the same 64-bit unsigned type on this ABI (LP64)
+    assert ctypes.sizeof(ctypes.c_size_t) == ctypes.sizeof(ctypes.c_uint64) == 8
+    return {ctypes.c_int: "i32", ctypes.c_int64: "i64", ctypes.c_uint64: "u64",
+            ctypes.c_size_t: "u64", ctypes.c_double: "f64"}[t]
+
+
+def test_binding_argument_kinds_match_the_header():
+    """Every prototype in the header against the binding's ctypes signature: same number of
+    arguments and, argument by argument, the same kind (32-bit int, 64-bit signed, 64-bit
+    unsigned, double, pointer), and the same return kind."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    src = re.sub(r"#.*", "", src)
+    protos = re.findall(r"([A-Za-z_][\w\s\*]*?)\b(q1m_\w+)\s*\(([^)]*)\)\s*;", src)
+    assert len(protos) == len(q1m.SIGNATURES)
+    for ret, name, params in protos:
+        restype, argtypes = q1m.SIGNATURES[name]
+        args = [a for a in params.split(",") if a.strip() and a.strip() != "void"]
+        assert len(args) == len(argtypes), name
+        for i, (a, t) in enumerate(zip(args, argtypes)):
+            assert _c_kind(a) == _ctypes_kind(t), (name, i, a, t)
+        assert _c_kind(ret) == _ctypes_kind(restype), (name, ret, restype)
