@@ -26,8 +26,10 @@
  *     or a malformed index list) are latched on the device and returned by q1m_status_poll().
  *   - Calls are thread-safe as long as concurrent calls use distinct workspaces/outputs.
  *   - head_dim is 64 or 128; n_q_heads is a multiple of n_kv_heads; (dca_chunk - local_window)
- *     and prefill_chunk are multiples of 128. Only sm_100a devices are supported; there is no
- *     CPU fallback.
+ *     and prefill_chunk are multiples of 128. Sparse mode takes at most 7 Q heads per KV head
+ *     (the estimator's 7 x 64 rows per group fill its tensor-memory accumulator), decode at
+ *     most 8; larger groups return Q1M_ERR_UNSUPPORTED. Only sm_100a devices are supported;
+ *     there is no CPU fallback.
  */
 #ifndef Q1M_H_
 #define Q1M_H_
