@@ -202,3 +202,20 @@ def test_binding_argument_kinds_match_the_header():
         for i, (a, t) in enumerate(zip(args, argtypes)):
             assert _c_kind(a) == _ctypes_kind(t), (name, i, a, t)
         assert _c_kind(ret) == _ctypes_kind(restype), (name, ret, restype)
+
+
+def test_group_size_limits(lib):
+    """Sparse mode takes at most 7 Q heads per KV head (the estimator's rows per group);
+    dense mode has no such limit; decode takes at most 8."""
+    w = C.SMALL_SPARSE
+    p = q1m.params(w)
+    assert lib.q1m_workspace_bytes(w.seq_len, 14, 2, 128, ctypes.byref(p)) > 0      # G = 7
+    assert lib.q1m_workspace_bytes(w.seq_len, 16, 2, 128, ctypes.byref(p)) == 0     # G = 8
+    st = lib.q1m_dca_sparse_prefill(1, 1, 1, 1, None, w.seq_len, 16, 2, 128, ctypes.byref(p),
+                                    256, 1 << 40, None)
+    assert st == -2 and "7 Q heads" in lib.q1m_last_error().decode()
+    pd = q1m.params(w.with_(vs_vertical=0, vs_slash=0))
+    assert lib.q1m_workspace_bytes(w.seq_len, 16, 2, 128, ctypes.byref(pd)) > 0     # dense
+    st = lib.q1m_dca_decode(1, 1, 1, 5, 1, 1, 128, 18, 2, 128, ctypes.byref(pd), 1, 1, None,
+                            256, 1 << 20, None)
+    assert st == -2, lib.q1m_last_error()
