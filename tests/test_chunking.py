@@ -32,3 +32,14 @@ def test_bounds_reject_bad_params():
         q1m.prefill_bounds(C.SMALL_SPARSE.with_(equal_cost_chunks=-1))
     with pytest.raises(q1m.Q1MError):
         q1m.prefill_bounds(C.SMALL_SPARSE.with_(prefill_chunk=100))
+
+
+@pytest.mark.parametrize("n,K", [((1 << 28) - 1, 7), ((1 << 27) + 77, 1000), (1 << 26, 1),
+                                 (5000, 4096), (129, 3)])
+def test_equal_cost_bounds_at_extreme_sizes(n, K):
+    """Near the library's largest sequence (2^28 rows: 128-bit cost arithmetic on the C side,
+    Python integers in the oracle) and with more chunks than blocks (dropped boundaries)."""
+    w = C.SMALL_SPARSE.with_(seq_len=n, equal_cost_chunks=K)
+    got = q1m.prefill_bounds(w)
+    assert got == list(O.prefill_chunks(w))
+    assert got[-1][1] == n and len(got) <= min(K, -(-n // 128))
