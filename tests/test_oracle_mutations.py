@@ -230,6 +230,39 @@ def _recall_squared(self, rows, h, sel):
     return res
 
 
+def _pattern_wrong_neighbour(i, j, cfg):
+    L = O.dca_len(cfg)
+    ci, cj = np.asarray(i) // L, np.asarray(j) // L
+    return np.where(ci == cj, O.INTRA, np.where(cj == ci - 2, O.SUCC, O.INTER))
+
+
+def _blocks_no_clamp(S, b, e, bs=O.BLOCK):
+    nkb = (e + bs - 1) // bs
+    r0, r1 = b * bs, min(b * bs + bs - 1, e - 1)
+    o = np.asarray(S, dtype=np.int64)
+    o = o[o <= r1]
+    lo, hi = (r0 - o) // bs, (r1 - o) // bs
+    cnt = np.zeros(nkb + 1, dtype=np.int64)
+    np.add.at(cnt, lo, 1)            # a negative start wraps to the end of the array
+    np.add.at(cnt, hi + 1, -1)
+    return np.cumsum(cnt)[:nkb] > 0
+
+
+def _top_unsorted(scores, budget):
+    scores = np.asarray(scores, dtype=np.float64)
+    n = scores.shape[0]
+    if budget >= n:
+        return np.arange(n, dtype=np.int64)
+    return np.lexsort((np.arange(n), -scores))[:budget].astype(np.int64)
+
+
+def _softmax_lse_base2(l):
+    m = np.max(l, axis=1, keepdims=True)
+    p = np.exp(l - m)
+    s = np.sum(p, axis=1, keepdims=True)
+    return p / s, (m + np.log2(s))[:, 0]
+
+
 MUTATIONS = [
     ("rope sign flipped", "rope", _rope_sign),
     ("rope pairs interleaved", "rope", _rope_interleaved),
@@ -260,6 +293,10 @@ MUTATIONS = [
     ("residual verticals stop one row early", "residual_verticals", _residual_cut_early),
     ("decode step leaves out the token's own key", "Oracle.decode_row", _decode_without_own_key),
     ("recall squared", "Oracle.recall_rows", _recall_squared),
+    ("successive pattern taken two chunks back", "dca_pattern", _pattern_wrong_neighbour),
+    ("slash block range not clamped at key block 0", "computed_blocks", _blocks_no_clamp),
+    ("selected indices not in ascending order", "top_budget", _top_unsorted),
+    ("log-sum-exp in base 2", "softmax_rows", _softmax_lse_base2),
 ]
 
 
