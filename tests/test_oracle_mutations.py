@@ -263,6 +263,24 @@ def _softmax_lse_base2(l):
     return p / s, (m + np.log2(s))[:, 0]
 
 
+def _estimator_single_row(s0, e, cfg):
+    return np.arange(e - 1, e)
+
+
+def _forced_on_top_of_budget(vert, slash, cfg):
+    S = O.top_budget(slash, cfg.vs_slash)
+    return (O.top_budget(vert, cfg.vs_vertical),
+            np.union1d(S, np.arange(min(cfg.vs_force_local, len(slash)))).astype(np.int64))
+
+
+def _intra_query_unwrapped(i, pattern, cfg):
+    if pattern == O.INTRA:
+        return np.asarray(i)
+    L, c = O.dca_len(cfg), cfg.dca_chunk
+    t = np.asarray(i) % L
+    return np.minimum(t + L, c - 1) if pattern == O.SUCC else np.full_like(t, c - 1)
+
+
 MUTATIONS = [
     ("rope sign flipped", "rope", _rope_sign),
     ("rope pairs interleaved", "rope", _rope_interleaved),
@@ -297,6 +315,9 @@ MUTATIONS = [
     ("slash block range not clamped at key block 0", "computed_blocks", _blocks_no_clamp),
     ("selected indices not in ascending order", "top_budget", _top_unsorted),
     ("log-sum-exp in base 2", "softmax_rows", _softmax_lse_base2),
+    ("estimator reads only the last row", "estimator_rows", _estimator_single_row),
+    ("forced diagonals added on top of the slash budget", "select_head", _forced_on_top_of_budget),
+    ("intra query at i instead of i mod L", "dca_query_position", _intra_query_unwrapped),
 ]
 
 
