@@ -263,6 +263,29 @@ def estimator_work(w) -> dict:
     return {"bytes": byts, "flops": flops, "exps": exps}
 
 
+# ex2 results per clock per SM on the multi-function units (measured on B200 with all SMs
+# busy: 15.99)
+MUFU_EXP_PER_CLK_PER_SM = 16
+
+
+def estimator_bounds(ew: dict, t_est: float, hbm_gbs: float, tensor_tflops: float, sms: int,
+                     sm_mhz: float) -> dict:
+    """The estimator's three bounds for its measured time t_est (s): HBM bytes, tensor FLOPs
+    and MUFU exponentials (peak = MUFU_EXP_PER_CLK_PER_SM x SMs x SM clock), each achieved and
+    as a fraction of its peak, and the HBM fraction the stage would reach if it ran exactly
+    at its exponential bound: the ceiling its arithmetic sets on the HBM fraction."""
+    exp_peak = MUFU_EXP_PER_CLK_PER_SM * sms * sm_mhz * 1e6      # exponentials per second
+    t_exp = ew["exps"] / exp_peak
+    return {"gbs": ew["bytes"] / t_est / 1e9,
+            "frac_hbm": ew["bytes"] / t_est / 1e9 / hbm_gbs,
+            "tflops": ew["flops"] / t_est / 1e12,
+            "frac_tensor": ew["flops"] / t_est / 1e12 / tensor_tflops,
+            "gexp_per_s": ew["exps"] / t_est / 1e9,
+            "exp_peak_gexp_per_s": exp_peak / 1e9,
+            "frac_exp": t_exp / t_est,
+            "frac_hbm_at_exp_bound": ew["bytes"] / t_exp / 1e9 / hbm_gbs}
+
+
 def dense_pairs(w) -> float:
     n = float(w.seq_len)
     return n * (n + 1) / 2 * w.n_q_heads
@@ -436,14 +459,13 @@ def main():
     if not w.dense and prof["estimate"][0] > 0:
         ew = estimator_work(w)
         t_est = prof["estimate"][0] / args.steps * 1e-3
-        estimator = {"ms_per_step": t_est * 1e3,
-                     "algorithmic_bytes": ew["bytes"], "gbs": ew["bytes"] / t_est / 1e9,
-                     "frac_hbm": ew["bytes"] / t_est / 1e9 / hbm,
-                     "tflops": ew["flops"] / t_est / 1e12,
-                     "frac_tensor": ew["flops"] / t_est / 1e12 / sustained,
-                     "gexp_per_s": ew["exps"] / t_est / 1e9,
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
+        mhz = clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0
+        estimator = {"ms_per_step": t_est * 1e3, "algorithmic_bytes": ew["bytes"],
+                     **estimator_bounds(ew, t_est, hbm, sustained, sms, float(mhz)),
                      "note": "two tcgen05 passes over the key prefix; at D=128 with 7 Q heads "
-                             "per KV head the tensor and exponential work, not HBM, bound it"}
+                             "per KV head the exponentials, not HBM, bound it: "
+                             "frac_hbm_at_exp_bound is the most HBM it can reach"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -94,3 +94,21 @@ def test_kernel_traffic_tracks_the_capture(tmp_path, monkeypatch):
     h = bench.kernel_source_hash()
     fake.write_text(f"traffic_per_launch_bytes: 123\nkernel_source_sha256: {h}\n")
     assert bench.kernel_traffic("7b-1m") == 123.0
+
+
+def test_estimator_bounds_identities_and_ceiling():
+    """The estimator's reported bounds are consistent (frac_hbm = frac_exp x the HBM
+    fraction at the exponential bound; frac_exp = achieved / peak exponential rate), and at
+    the 7B shape its exponentials cap its HBM fraction near 0.45: per key and chunk it reads
+    2 passes x 4 KV heads x 128 x 2 bytes = 2,048 bytes and writes 2 x 28 x 4 = 224 bytes of
+    scores, and computes 2 x 64 x 28 = 3,584 exponentials; 16 exponentials per clock on 148
+    SMs at 1,965 MHz against 6,538.9 GB/s give 2272 / 3584 x 4.653e12 / 6.5389e12 = 0.451."""
+    import bench
+    from synth import configs as C
+    ew = bench.estimator_work(C.L7B_1M)
+    b = bench.estimator_bounds(ew, 27.3e-3, 6538.9, 1402.6, 148, 1965.0)
+    assert abs(b["frac_hbm"] - b["frac_exp"] * b["frac_hbm_at_exp_bound"]) < 1e-12
+    assert abs(b["frac_exp"] - b["gexp_per_s"] / b["exp_peak_gexp_per_s"]) < 1e-12
+    assert abs(b["exp_peak_gexp_per_s"] - 16 * 148 * 1.965) < 1e-6
+    assert 0.445 < b["frac_hbm_at_exp_bound"] < 0.455, b["frac_hbm_at_exp_bound"]
+    assert 0.0 < b["frac_exp"] < 1.0 and 0.0 < b["frac_hbm"] < b["frac_hbm_at_exp_bound"]
