@@ -495,6 +495,11 @@ def check_decode_row() -> float:
             err = max(err, float(np.max(np.abs(got - ref))), abs(lse - (mx + math.log(w.sum()))))
     ones = O.Oracle(q, k, np.ones_like(v), cfg)
     err = max(err, float(np.max(np.abs(ones.decode_row(cfg.seq_len - 1, 1)[0] - 1.0))))
+    # the decode step of the token at pos is row pos of the dense prefill (reading C12)
+    for pos in (0, L, 2 * L + 5, cfg.seq_len - 1):
+        o, l = orc.attend_rows(np.array([pos]), 2, O.ChunkSelection(0, cfg.seq_len))
+        d, dl = orc.decode_row(pos, 2)
+        err = max(err, float(np.max(np.abs(o[0] - d))), abs(float(l[0]) - dl))
     return err
 
 
