@@ -441,6 +441,25 @@ def check_recall() -> float:
     return err if low < 0.9 else float("inf")
 
 
+def check_fixed_chunks() -> bool:
+    """Fixed-size chunked prefill (the pages' --max-num-batched-tokens): hand-worked chunk
+    lists, and the layer's selections follow them (each selection's [s0, e) is a chunk and
+    its estimator rows are that chunk's last rows)."""
+    cases = {(300, 128): [(0, 128), (128, 256), (256, 300)], (256, 128): [(0, 128), (128, 256)],
+             (5, 128): [(0, 5)], (129, 128): [(0, 128), (128, 129)]}
+    ok = True
+    for (n, P), want in cases.items():
+        ok &= list(O.prefill_chunks(tiny(seq_len=n, prefill_chunk=P))) == want
+    cfg = tiny(seq_len=300, dca_chunk=80, local_window=16, vs_vertical=4, vs_slash=10,
+               vs_force_local=2, prefill_chunk=128)
+    q, k, v = rand_qkv(cfg, 31)
+    sels = O.Oracle(q, k, v, cfg).run()[2]
+    ok &= [(s.s0, s.e) for s in sels] == cases[(300, 128)]
+    for s in sels:
+        ok &= s.est_lse.shape[1] == min(cfg.vs_last_q, s.e - s.s0)
+    return bool(ok)
+
+
 def check_equal_cost_chunks() -> int:
     """The equal-cost chunking against the hand-worked fixture and its invariants: chunks
     tile [0, n) in 128-row blocks, there are at most K, and each chunk's dense cost is within

@@ -37,6 +37,7 @@ def _all_checks():
     res["recall"] = C.check_recall() < 1e-12
     res["key_order"] = C.check_key_order_invariance() < 1e-12
     res["residual"] = C.check_residual_verticals()
+    res["fixed_chunks"] = C.check_fixed_chunks()
     return res
 
 
@@ -281,6 +282,14 @@ def _intra_query_unwrapped(i, pattern, cfg):
     return np.minimum(t + L, c - 1) if pattern == O.SUCC else np.full_like(t, c - 1)
 
 
+def _fixed_chunks_one_row_longer(cfg):
+    if getattr(cfg, "equal_cost_chunks", 0) > 0:
+        yield from O.equal_cost_chunks(cfg.seq_len, cfg.equal_cost_chunks)
+        return
+    for s0 in range(0, cfg.seq_len, cfg.prefill_chunk + 1):
+        yield s0, min(cfg.seq_len, s0 + cfg.prefill_chunk + 1)
+
+
 MUTATIONS = [
     ("rope sign flipped", "rope", _rope_sign),
     ("rope pairs interleaved", "rope", _rope_interleaved),
@@ -318,6 +327,7 @@ MUTATIONS = [
     ("estimator reads only the last row", "estimator_rows", _estimator_single_row),
     ("forced diagonals added on top of the slash budget", "select_head", _forced_on_top_of_budget),
     ("intra query at i instead of i mod L", "dca_query_position", _intra_query_unwrapped),
+    ("fixed prefill chunks one row longer", "prefill_chunks", _fixed_chunks_one_row_longer),
 ]
 
 

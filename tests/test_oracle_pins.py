@@ -92,3 +92,7 @@ def test_key_order_invariance():
 
 def test_residual_verticals_complete_the_attended_set():
     assert C.check_residual_verticals()
+
+
+def test_fixed_prefill_chunks():
+    assert C.check_fixed_chunks()
