@@ -28,8 +28,10 @@
  *   - head_dim is 64 or 128; n_q_heads is a multiple of n_kv_heads; (dca_chunk - local_window)
  *     and prefill_chunk are multiples of 128. Sparse mode takes at most 7 Q heads per KV head
  *     (the estimator's 7 x 64 rows per group fill its tensor-memory accumulator), decode at
- *     most 8; larger groups return Q1M_ERR_UNSUPPORTED. Only sm_100a devices are supported;
- *     there is no CPU fallback.
+ *     most 8; larger groups return Q1M_ERR_UNSUPPORTED. A prefill chunk holds at most
+ *     Q1M_MAX_CHUNK_QUERY_BLOCKS query blocks of 128 rows; a layer or attention call with a
+ *     larger chunk returns Q1M_ERR_UNSUPPORTED before anything is launched. Only sm_100a
+ *     devices are supported; there is no CPU fallback.
  */
 #ifndef Q1M_H_
 #define Q1M_H_
@@ -54,6 +56,10 @@ typedef enum {
 } q1m_status;
 
 typedef enum { Q1M_BF16 = 0, Q1M_F32 = 1 } q1m_dtype;
+
+/* Largest prefill chunk the attention stage takes, in 128-row query blocks (4,194,304 rows):
+ * its work-unit sort keeps 3 x ceil(blocks / 2) costs in one CTA's shared memory. */
+#define Q1M_MAX_CHUNK_QUERY_BLOCKS 32768
 
 /* Layer parameters. Mirrors the pages' deployment knobs: dca_chunk / local_window (DCA),
  * yarn_s (YaRN ratio s), prefill_chunk (--max-num-batched-tokens) and the vertical-slash
@@ -250,7 +256,9 @@ q1m_status q1m_block_sparse_attn(const uint16_t* qv, int64_t ld_rows, const uint
  * rejected with Q1M_ERR_UNSUPPORTED before anything is launched. The call allocates nothing
  * (no cudaMalloc, cudaFree or allocating library routine). The first call on each device
  * looks up the array's device address (cudaGetSymbolAddress) with that device current, so
- * make that first call before any stream capture. All calls share the one array, and each
+ * make that first call before any stream capture; the address is looked up again when the
+ * device's context has changed (after cudaDeviceReset), and that call, too, must come
+ * before any capture. All calls share the one array, and each
  * call rewrites every entry it reads; calls that can overlap on the GPU (different
  * streams, or devices sharing it) race on it and must be serialised by the caller. */
 #define Q1M_NOALLOC_UNITS 16384

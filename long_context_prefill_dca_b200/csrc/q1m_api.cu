@@ -205,6 +205,16 @@ int64_t max_chunk_rows(int64_t n, const q1m_params* p) {
   return mx;
 }
 
+// The attention stage sorts a chunk's work units in one CTA's shared memory, so a prefill
+// chunk may hold at most Q1M_MAX_CHUNK_QUERY_BLOCKS query blocks.
+q1m_status check_chunks(int64_t n, const q1m_params* p) {
+  const int64_t rows = max_chunk_rows(n, p);
+  if (rows > (int64_t)128 * Q1M_MAX_CHUNK_QUERY_BLOCKS)
+    return fail(Q1M_ERR_UNSUPPORTED, "a prefill chunk of %lld rows exceeds %d query blocks",
+                (long long)rows, Q1M_MAX_CHUNK_QUERY_BLOCKS);
+  return Q1M_OK;
+}
+
 float view_scale(const q1m_params* p, int d) {
   const double s = p->yarn_s;
   double inv_t = 1.0;
@@ -508,6 +518,7 @@ q1m_status run_attn_d(const uint16_t* qv, int64_t ld_rows, const uint16_t* k_rot
   a.n_units = units;
   a.aligned = deterministic_on() ? 0 : 1;
   const int U = 3 * a.npair;
+  Q1M_CUDA(cudaFuncSetAttribute(k3_units_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, U * 4));
   k3_units_kernel<<<1, 1024, (size_t)U * 4, st>>>(s0, a.nqb, a.L, units + 8, units);
   Q1M_LAUNCHED();
   CUtensorMap mq, mk, mv;
@@ -615,12 +626,12 @@ const char* q1m_version(void) { return "q1m 0.1 (sm_100a)"; }
 const char* q1m_last_error(void) { return t_err.c_str(); }
 
 size_t q1m_workspace_bytes(int64_t n, int hq, int hkv, int d, const q1m_params* p) {
-  if (check_shape(n, hq, hkv, d, p) != Q1M_OK) return 0;
+  if (check_shape(n, hq, hkv, d, p) != Q1M_OK || check_chunks(n, p) != Q1M_OK) return 0;
   return layout(n, hq, hkv, d, p).total;
 }
 
 size_t q1m_host_workspace_bytes(int64_t n, int hq, int hkv, int d, const q1m_params* p) {
-  if (check_shape(n, hq, hkv, d, p) != Q1M_OK) return 0;
+  if (check_shape(n, hq, hkv, d, p) != Q1M_OK || check_chunks(n, p) != Q1M_OK) return 0;
   const size_t ein = p->in_dtype == Q1M_BF16 ? 2 : 4, eout = p->out_dtype == Q1M_BF16 ? 2 : 4;
   return align_up((size_t)n * hq * d * ein) + 2 * align_up((size_t)n * hkv * d * ein) +
          align_up((size_t)n * hq * d * eout) + align_up((size_t)n * hq * 4) +
@@ -721,6 +732,9 @@ q1m_status q1m_block_sparse_attn(const uint16_t* qv, int64_t ld_rows, const uint
   if (mask && (!cnt || (p->vs_vertical > 0 && !resid))) return fail(Q1M_ERR_INVALID, "mask without counts/residuals");
   if (s0 < 0 || e <= s0 || s0 % 128 || ld_rows < e - s0 || ld_rows % 128 || ld_tokens < e || ld_tokens % 128)
     return fail(Q1M_ERR_INVALID, "bad range");
+  if ((e - s0 + 127) / 128 > Q1M_MAX_CHUNK_QUERY_BLOCKS)
+    return fail(Q1M_ERR_UNSUPPORTED, "a chunk of %lld query blocks exceeds %d", (long long)((e - s0 + 127) / 128),
+                Q1M_MAX_CHUNK_QUERY_BLOCKS);
   if (scratch_bytes < q1m_attn_scratch_bytes(s0, e, hq, d)) return fail(Q1M_ERR_WORKSPACE, "attention scratch too small");
   if (reinterpret_cast<uintptr_t>(scratch) & 3) return fail(Q1M_ERR_INVALID, "scratch misaligned");
   Dev dev;
@@ -778,6 +792,7 @@ static q1m_status prefill_range(const void* q, const void* k, const void* v, voi
                                 const q1m_params* p, int64_t first_chunk, int64_t last_chunk,
                                 void* ws, size_t ws_bytes, void* stream, ChunkHooks* hooks) {
   Q1M_TRY(check_shape(n, hq, hkv, d, p));
+  Q1M_TRY(check_chunks(n, p));
   if (first_chunk < 0 || last_chunk < first_chunk) return fail(Q1M_ERR_INVALID, "bad chunk range");
   if (!q || !k || !v || !out || !ws) return fail(Q1M_ERR_INVALID, "NULL pointer");
   if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(Q1M_ERR_INVALID, "workspace must be 256-byte aligned");
@@ -931,6 +946,7 @@ q1m_status q1m_dca_sparse_prefill_host(const void* q_h, const void* k_h, const v
                                        float* lse_h, int64_t n, int hq, int hkv, int d,
                                        const q1m_params* p, void* ws, size_t ws_bytes, void* stream) {
   Q1M_TRY(check_shape(n, hq, hkv, d, p));
+  Q1M_TRY(check_chunks(n, p));
   if (!q_h || !k_h || !v_h || !out_h || !ws) return fail(Q1M_ERR_INVALID, "NULL pointer");
   if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(Q1M_ERR_INVALID, "workspace must be 256-byte aligned");
   if (ws_bytes < q1m_host_workspace_bytes(n, hq, hkv, d, p)) return fail(Q1M_ERR_WORKSPACE, "host-path workspace too small");
@@ -977,10 +993,10 @@ q1m_status q1m_dca_decode(const void* q, const void* k, const void* v, int64_t p
                           void* scratch, size_t scratch_bytes, void* stream) {
   if (pos < 0) return fail(Q1M_ERR_INVALID, "pos must be >= 0");
   Q1M_TRY(check_shape(pos + 1, hq, hkv, d, p));
+  if (hq / hkv > 8) return fail(Q1M_ERR_UNSUPPORTED, "decode supports at most 8 Q heads per KV head");
   if (!q || !k || !v || !k_rot || !v16 || !table || !out || !scratch) return fail(Q1M_ERR_INVALID, "NULL pointer");
   if (ld_tokens <= pos || ld_tokens % 128) return fail(Q1M_ERR_INVALID, "ld_tokens must be a multiple of 128 and > pos");
   if ((int64_t)hkv * ld_tokens >= ((int64_t)1 << 31)) return fail(Q1M_ERR_UNSUPPORTED, "n_kv_heads * ld_tokens too large");
-  if (hq / hkv > 8) return fail(Q1M_ERR_UNSUPPORTED, "decode supports at most 8 Q heads per KV head");
   if (scratch_bytes < q1m_dca_decode_scratch_bytes(hq, d)) return fail(Q1M_ERR_WORKSPACE, "decode scratch too small");
   if (reinterpret_cast<uintptr_t>(scratch) & 255) return fail(Q1M_ERR_INVALID, "scratch must be 256-byte aligned");
   Dev dev;
@@ -1150,23 +1166,53 @@ extern "C" q1m_status q1m_selftest_wait_timeout(uint64_t cycles, void* stream) {
 // =============================================================================================
 namespace {
 static __device__ __align__(256) int32_t g_noalloc_units[Q1M_NOALLOC_UNITS];
+static_assert(3 * (Q1M_NOALLOC_MAX_QUERY_BLOCKS + 1) / 2 + 8 <= Q1M_NOALLOC_UNITS,
+              "the static work list holds the largest chunk it admits");
+static_assert(Q1M_NOALLOC_MAX_QUERY_BLOCKS <= Q1M_MAX_CHUNK_QUERY_BLOCKS, "within the stage limit");
 std::mutex g_noalloc_mu;
 constexpr int kMaxDevices = 64;
-int32_t* g_noalloc_ptr[kMaxDevices] = {};
+struct NoallocSlot {
+  void* ctx = nullptr;       // the device's context when ptr was looked up
+  int32_t* ptr = nullptr;
+};
+NoallocSlot g_noalloc_slot[kMaxDevices];
 
-// Device address of g_noalloc_units on the current device (looked up once per device; the
-// array's name in host code is only a stand-in for the symbol).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  return fn;
+}
+
+// Device address of g_noalloc_units on the current device. In host code the array's name is
+// only a stand-in for the symbol, so the address is looked up with cudaGetSymbolAddress the
+// first time a device is used, and again whenever that device's context differs from the one
+// the address was taken in (a cudaDeviceReset reloads the module at another address).
 q1m_status noalloc_units(int32_t** out) {
   int dev = 0;
   Q1M_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return fail(Q1M_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  auto get = ctx_get_current();
+  if (!get) return fail(Q1M_ERR_CUDA, "cuCtxGetCurrent unavailable");
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return fail(Q1M_ERR_CUDA, "cuCtxGetCurrent failed");
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoallocSlot& sl = g_noalloc_slot[dev];
+  if (!sl.ptr || !ctx || sl.ctx != static_cast<void*>(ctx)) {
     void* ptr = nullptr;
-    Q1M_CUDA(cudaGetSymbolAddress(&ptr, g_noalloc_units));
-    g_noalloc_ptr[dev] = static_cast<int32_t*>(ptr);
+    Q1M_CUDA(cudaGetSymbolAddress(&ptr, g_noalloc_units));   // binds the context if needed
+    if (get(&ctx) != CUDA_SUCCESS || !ctx) return fail(Q1M_ERR_CUDA, "no current CUDA context");
+    sl.ptr = static_cast<int32_t*>(ptr);
+    sl.ctx = ctx;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = sl.ptr;
   return Q1M_OK;
 }
 }  // namespace
@@ -1176,16 +1222,18 @@ extern "C" q1m_status q1m_block_sparse_attn_noalloc(
     int64_t ld_tokens, const uint32_t* mask, const int32_t* resid, const int32_t* cnt, int64_t s0,
     int64_t e, int hq, int hkv, int d, const q1m_params* p, float* o_part, float* lse_part,
     void* stream) {
+  // the size limit first: a chunk the static list cannot hold is refused whatever else is passed
+  if (e > s0 && s0 >= 0) {
+    const int64_t nqb = (e - s0 + 127) / 128;
+    if (nqb > Q1M_NOALLOC_MAX_QUERY_BLOCKS)
+      return fail(Q1M_ERR_UNSUPPORTED, "chunk of %lld query blocks exceeds the static work list (%d blocks)",
+                  (long long)nqb, Q1M_NOALLOC_MAX_QUERY_BLOCKS);
+  }
   Q1M_TRY(check_shape(e > 0 ? e : 1, hq, hkv, d, p));
   if (!qv || !k_rot || !v16 || !o_part || !lse_part) return fail(Q1M_ERR_INVALID, "NULL pointer");
   if (mask && (!cnt || (p->vs_vertical > 0 && !resid))) return fail(Q1M_ERR_INVALID, "mask without counts/residuals");
   if (s0 < 0 || e <= s0 || s0 % 128 || ld_rows < e - s0 || ld_rows % 128 || ld_tokens < e || ld_tokens % 128)
     return fail(Q1M_ERR_INVALID, "bad range");
-  const int64_t nqb = (e - s0 + 127) / 128;
-  if (nqb > Q1M_NOALLOC_MAX_QUERY_BLOCKS ||
-      q1m_attn_scratch_bytes(s0, e, hq, d) > sizeof(int32_t) * Q1M_NOALLOC_UNITS)
-    return fail(Q1M_ERR_UNSUPPORTED, "chunk of %lld query blocks exceeds the static work list (%d blocks)",
-                (long long)nqb, Q1M_NOALLOC_MAX_QUERY_BLOCKS);
   Dev dev;
   Q1M_TRY(device_info(&dev));
   int32_t* units = nullptr;

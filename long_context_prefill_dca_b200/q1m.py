@@ -15,6 +15,10 @@ Q1M_OK = 0
 STATUS = {0: "Q1M_OK", -1: "Q1M_ERR_INVALID", -2: "Q1M_ERR_UNSUPPORTED", -3: "Q1M_ERR_WORKSPACE",
           -4: "Q1M_ERR_CUDA", -5: "Q1M_ERR_TIMEOUT", -6: "Q1M_ERR_RANGE"}
 BF16, F32 = 0, 1
+# size limits, as include/q1m.h defines them
+MAX_CHUNK_QUERY_BLOCKS = 32768      # Q1M_MAX_CHUNK_QUERY_BLOCKS
+NOALLOC_UNITS = 16384               # Q1M_NOALLOC_UNITS
+NOALLOC_MAX_QUERY_BLOCKS = 10916    # Q1M_NOALLOC_MAX_QUERY_BLOCKS
 
 c_i32, c_i64, c_u64, c_dbl = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_double
 c_size, c_vp, c_int = ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int

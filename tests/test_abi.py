@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from long_context_prefill_dca_b200 import build, q1m
 from synth import configs as C
@@ -36,6 +37,15 @@ def test_version(lib):
     assert "sm_100a" in q1m.version()
 
 
+# Tests that pass stand-in pointers (small integers, not device memory) to reach a check that
+# follows the NULL check. With no GPU present the library cannot launch anything, so a check
+# that went missing fails the test instead of touching memory; on a machine with a GPU they
+# are skipped.
+host_only = pytest.mark.skipif(torch.cuda.is_available(),
+                               reason="passes stand-in device pointers; host-only")
+
+
+@host_only
 @pytest.mark.parametrize("field,value,code", [
     ("dca_chunk", 1000, -2),         # c - w not a multiple of 128
     ("local_window", -1, -1),
@@ -54,6 +64,7 @@ def test_invalid_params_rejected_without_launch(lib, field, value, code):
     assert lib.q1m_last_error().decode()
 
 
+@host_only
 def test_bad_shapes_rejected(lib):
     w = C.SMALL_SPARSE
     p = q1m.params(w)
@@ -66,8 +77,9 @@ def test_bad_shapes_rejected(lib):
     st = lib.q1m_dca_sparse_prefill(1, 1, 1, 1, None, w.seq_len, 4, 2, 128, ctypes.byref(p),
                                     256, 10, None)
     assert st == -3          # workspace too small
-    st = lib.q1m_dca_sparse_prefill(1, 1, 1, 1, None, w.seq_len, 16, 2, 128, ctypes.byref(p),
-                                    256, 1 << 40, None)
+    # NULL device pointers: nothing here can reach a launch, whatever the order of the checks
+    st = lib.q1m_dca_sparse_prefill(None, None, None, None, None, w.seq_len, 16, 2, 128,
+                                    ctypes.byref(p), None, 1 << 40, None)
     assert st == -2          # 8 Q heads per KV head exceeds the estimator
 
 
@@ -77,6 +89,7 @@ def test_workspace_sizes_monotone(lib):
     assert 0 < small < big < 40 * 2**30
 
 
+@host_only
 def test_decode_validates_before_launch():
     """q1m_dca_decode rejects bad arguments on the host, before touching the device."""
     import ctypes
@@ -98,6 +111,7 @@ def test_decode_validates_before_launch():
                               None, 256, nb, None) == -1                       # NULL pointer
 
 
+@host_only
 def test_chunk_range_validated():
     import ctypes
     from long_context_prefill_dca_b200 import q1m
@@ -211,11 +225,42 @@ def test_group_size_limits(lib):
     p = q1m.params(w)
     assert lib.q1m_workspace_bytes(w.seq_len, 14, 2, 128, ctypes.byref(p)) > 0      # G = 7
     assert lib.q1m_workspace_bytes(w.seq_len, 16, 2, 128, ctypes.byref(p)) == 0     # G = 8
-    st = lib.q1m_dca_sparse_prefill(1, 1, 1, 1, None, w.seq_len, 16, 2, 128, ctypes.byref(p),
-                                    256, 1 << 40, None)
+    st = lib.q1m_dca_sparse_prefill(None, None, None, None, None, w.seq_len, 16, 2, 128,
+                                    ctypes.byref(p), None, 1 << 40, None)
     assert st == -2 and "7 Q heads" in lib.q1m_last_error().decode()
     pd = q1m.params(w.with_(vs_vertical=0, vs_slash=0))
     assert lib.q1m_workspace_bytes(w.seq_len, 16, 2, 128, ctypes.byref(pd)) > 0     # dense
-    st = lib.q1m_dca_decode(1, 1, 1, 5, 1, 1, 128, 18, 2, 128, ctypes.byref(pd), 1, 1, None,
-                            256, 1 << 20, None)
+    st = lib.q1m_dca_decode(None, None, None, 5, None, None, 128, 18, 2, 128, ctypes.byref(pd),
+                            None, None, None, None, 1 << 20, None)
     assert st == -2, lib.q1m_last_error()
+
+
+def test_header_limits_match_the_binding():
+    """The size limits #defined in the header are the binding's constants."""
+    src = open(HEADER).read()
+    defs = dict(re.findall(r"#define\s+(Q1M_\w+)\s+(\d+)", src))
+    assert int(defs["Q1M_MAX_CHUNK_QUERY_BLOCKS"]) == q1m.MAX_CHUNK_QUERY_BLOCKS
+    assert int(defs["Q1M_NOALLOC_UNITS"]) == q1m.NOALLOC_UNITS
+    assert int(defs["Q1M_NOALLOC_MAX_QUERY_BLOCKS"]) == q1m.NOALLOC_MAX_QUERY_BLOCKS
+    # the static list holds the largest chunk it admits, and one block more does not fit
+    units = lambda nqb: 3 * (nqb + 1) // 2 + 8
+    assert units(q1m.NOALLOC_MAX_QUERY_BLOCKS) <= q1m.NOALLOC_UNITS < units(q1m.NOALLOC_MAX_QUERY_BLOCKS + 1)
+
+
+def test_chunk_size_limit(lib):
+    """A prefill chunk above Q1M_MAX_CHUNK_QUERY_BLOCKS query blocks is refused by the
+    workspace query (0 bytes) and by the layer call before anything is launched; every device
+    pointer is NULL, so a changed check order would be refused by the NULL check instead."""
+    w = C.SMALL_DENSE_D128
+    big = 128 * q1m.MAX_CHUNK_QUERY_BLOCKS
+    ok = q1m.params(w.with_(seq_len=big, prefill_chunk=big))
+    assert lib.q1m_workspace_bytes(big, 1, 1, 64, ctypes.byref(ok)) > 0
+    p = q1m.params(w.with_(seq_len=big + 128, prefill_chunk=big + 128))
+    assert lib.q1m_workspace_bytes(big + 128, 1, 1, 64, ctypes.byref(p)) == 0
+    assert lib.q1m_host_workspace_bytes(big + 128, 1, 1, 64, ctypes.byref(p)) == 0
+    st = lib.q1m_dca_sparse_prefill(None, None, None, None, None, big + 128, 1, 1, 64,
+                                    ctypes.byref(p), None, 0, None)
+    assert st == -2 and "exceeds" in lib.q1m_last_error().decode()
+    # the same rows in chunks of the largest size are fine
+    p2 = q1m.params(w.with_(seq_len=big + 128, prefill_chunk=big))
+    assert lib.q1m_workspace_bytes(big + 128, 1, 1, 64, ctypes.byref(p2)) > 0
