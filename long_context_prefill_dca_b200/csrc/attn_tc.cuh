@@ -46,13 +46,14 @@ constexpr float K3_RESCALE_THRESHOLD = 8.0f;
 // rest on the MUFU; measured on B200 with both slots' softmax warps active, 2 to 4 of 8 on the
 // FMA pipe made the kernel 10-35% slower, so the default is 0
 constexpr int K3_POLY_PAIRS_OF_8 = 0;
-// P overwrites the first half of S, so the slot's next QK^T (which writes S) must not
-// overtake the PV MMA that reads P. tcgen05.mma operations issued by one thread execute in
-// issue order, and a later MMA's accumulator writes follow an earlier MMA's operand reads,
-// so no wait is needed between them; measured on B200 the explicit wait (a commit and an
-// mbarrier round trip per tile) costs 11% of the cycles and the outputs are bit-identical
-// either way. Setting this to true restores the explicit wait.
-constexpr bool K3_WAIT_PV_BEFORE_QK = false;
+// P overwrites the first half of S (columns 0..63), so the slot's next QK^T must not write
+// S before the PV MMA that reads P has completed. The PTX ISA guarantees that two
+// tcgen05.mma execute in issue order only when they share the accumulator and the shape
+// (its tcgen05 "pipelined instructions" pairs); QK^T (accumulator S) and PV (accumulator O)
+// do not, so the MMA warp waits for the PV's commit before it issues the next QK^T of the
+// slot. Measured on B200 this wait costs 3.5-4% of the kernel's time; issuing QK^T as two
+// N = 64 halves, the half clear of P first, to hide it was 15-17% slower (N = 64 MMAs re-read
+// the Q tile from shared memory for each half).
 
 struct K3Args {
   int64_t s0, e;
@@ -356,7 +357,7 @@ __device__ __forceinline__ bool k3_pv(K3Smem<D>& sm, const K3Desc& dsc, K3Slot& 
     for (int kk = 0; kk < 8; ++kk)   // 16 keys = 16 rows of 128 B per step (2048 B, >> 4 = 128)
       mma_ts(o_t, p_t + kk * 8u, vd + (uint64_t)(kk * 128), IDESC_PV,
              (sl.o_started || kk > 0) ? 1u : 0u);
-    // P lives in S's columns: the slot's next QK^T may overwrite them only after this PV
+    // P lives in S's columns 0..63: the slot's next QK^T is issued only after this commit
     mma_commit(&sm.pv_done[S]);
     if (sl.pend_last) mma_commit(&sm.o_done[S]);
     if (u == 0) mma_commit(&sm.v_empty[vst]);
@@ -381,9 +382,10 @@ __device__ __forceinline__ bool k3_qk(K3Smem<D>& sm, const K3Desc& dsc, K3Slot& 
     first = false;
     tc_fence_after();
   }
-  if (K3_WAIT_PV_BEFORE_QK && sl.pvd_waited < sl.pvd_issued) {
+  if (sl.pvd_waited < sl.pvd_issued) {   // the slot's previous PV still reads P (S columns)
     if (!mbar_wait_warp(&sm.pv_done[S], sl.pvd_waited & 1)) return false;
     ++sl.pvd_waited;
+    tc_fence_after();
   }
   --rem;
   const bool last = rem == 0;
