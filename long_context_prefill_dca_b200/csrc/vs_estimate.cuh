@@ -24,7 +24,9 @@ namespace q1m {
 
 constexpr int EA_THREADS = 192;   // warps 0-3 softmax, 4 loader, 5 MMA
 constexpr int EA_NK = 2;
-constexpr int EB_THREADS = 320;   // warps 0-7 epilogue (2 groups), 8 loader, 9 MMA
+constexpr int EB_THREADS = 576;   // warps 0-15 epilogue (4 groups), 16 loader, 17 MMA
+constexpr int EB_GROUPS = 4;      // epilogue groups of 4 warps (one per TMEM lane quarter)
+constexpr int EB_STEP = 16;       // est rows per epilogue step
 constexpr int EB_NK = 2;
 constexpr int EB_MAX_ROWS = 448;
 constexpr int EB_U = 192;         // offsets per key tile (64 + 128 - 1 used)
@@ -211,8 +213,8 @@ struct EBSmem {
   static constexpr int EST = EB_MAX_ROWS * D * 2;
   alignas(1024) uint8_t est[EST];         // est rows, [half][row][64 halfs] swizzled
   alignas(1024) uint8_t k[EB_NK][TILE];
-  float pbuf[2][32][128];                 // per epilogue group: 32 rows x 128 keys
-  float lse[2][EB_MAX_ROWS];              // per epilogue group
+  float pbuf[EB_GROUPS][EB_STEP][128];    // per epilogue group: EB_STEP rows x 128 keys
+  float lse[EB_GROUPS][EB_MAX_ROWS];      // per epilogue group
   uint64_t k_full[EB_NK], k_empty[EB_NK], e_full, e_empty, acc_full, acc_free, drain;
   uint32_t tmem_base;
 };
@@ -231,11 +233,12 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < EB_NK; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 1); }
     mbar_init(&sm.e_full, 1); mbar_init(&sm.e_empty, 1);
-    mbar_init(&sm.acc_full, 1); mbar_init(&sm.acc_free, 256);
+    mbar_init(&sm.acc_full, 1); mbar_init(&sm.acc_free, 32 * 4 * EB_GROUPS);
     mbar_init(&sm.drain, 1);
     fence_mbar_init();
   }
-  if (w == 9) { tmem_alloc(&sm.tmem_base, 512); tmem_relinquish(); }
+  constexpr int W_LOAD = 4 * EB_GROUPS, W_MMA = 4 * EB_GROUPS + 1;
+  if (w == W_MMA) { tmem_alloc(&sm.tmem_base, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -243,7 +246,7 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
   // the est-row operand is [half][row] with rows of 128 bytes; a 64-row-aligned row offset
   // keeps the 1024-byte swizzle atoms intact
   const uint32_t EST_HALF = (uint32_t)EB_MAX_ROWS * 128u;
-  if (w == 8) {
+  if (w == W_LOAD) {
     if (lane_id() == 0) {
       bool ok = true;
       int key_cur = -1, en = 0;
@@ -272,7 +275,7 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
       }
       if (!ok) { const long long c0 = clock64(); while (clock64() - c0 < 2000000) __nanosleep(1000); }
     }
-  } else if (w == 9) {
+  } else if (w == W_MMA) {
     if (lane_id() == 0) {
       bool ok = true;
       int key_cur = -1, en = 0;
@@ -312,7 +315,8 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
       mbar_wait(&sm.drain, 0);
     }
   } else {
-    // epilogue: group eg = w / 4 handles heads hh = eg, eg + 2, ...; thread owns key lane kl
+    // epilogue: group eg = w / 4 handles heads hh = eg, eg + EB_GROUPS, ...; thread owns key
+    // lane kl (its warp's TMEM lane quarter)
     const int eg = w >> 2;
     const int kl = 32 * (w & 3) + (int)lane_id();
     const uint32_t lb = tb + ((32u * (w & 3)) << 16);
@@ -332,15 +336,15 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
       if (!ok) break;
       tc_fence_after();
       const int64_t j = (int64_t)kt * 128 + kl;              // this thread's key
-      for (int hh = eg; hh < a.G; hh += 2) {
+      for (int hh = eg; hh < a.G; hh += EB_GROUPS) {
         float vsum = 0.f;
         float acc0 = 0.f, acc1 = 0.f;   // slash sums for U = kl and U = kl + 128
-        for (int rh = 0; rh < 2; ++rh) {
-          uint32_t rr[32];
-          tmem_ld32(lb + (uint32_t)(hh * 64 + rh * 32), rr);
+        for (int rh = 0; rh < 64 / EB_STEP; ++rh) {
+          uint32_t rr[EB_STEP];
+          tmem_ld16(lb + (uint32_t)(hh * 64 + rh * EB_STEP), rr);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int r = rh * 32 + c;
+          for (int c = 0; c < EB_STEP; ++c) {
+            const int r = rh * EB_STEP + c;
             const int64_t i = a.r_lo + r;
             float p = 0.f;
             if (r < nR && j <= i) p = ex2(__uint_as_float(rr[c]) - sm.lse[eg][hh * 64 + r]);
@@ -348,10 +352,10 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
             sm.pbuf[eg][c][kl] = p;
           }
           named_bar_sync(1 + eg, 128);
-          // U = 32 rh + c - k + 127 for row c of this half and key k of the tile
+          // U = EB_STEP rh + c - k + 127 for row c of this step and key k of the tile
 #pragma unroll 4
-          for (int c = 0; c < 32; ++c) {
-            const int k0 = 32 * rh + c + 127 - kl;
+          for (int c = 0; c < EB_STEP; ++c) {
+            const int k0 = EB_STEP * rh + c + 127 - kl;
             if (k0 >= 0 && k0 < 128) acc0 += sm.pbuf[eg][c][k0];
             const int k1 = k0 - 128;
             if (k1 >= 0 && k1 < 128) acc1 += sm.pbuf[eg][c][k1];
@@ -371,7 +375,7 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (w == 9) { __syncwarp(); tmem_dealloc(tb, 512); }
+  if (w == W_MMA) { __syncwarp(); tmem_dealloc(tb, 512); }
 }
 
 // slash[h][o] = sum of the (at most two) key tiles' partials that contain offset o, in
