@@ -1,10 +1,16 @@
 """Full-size workloads (128K, 256K, 1M and the ragged 1.01M layer), in the launch
 configuration the benchmark times, checked against the fp64 oracle on sampled rows.
 
-For each workload: the GPU runs every prefill chunk stage by stage; for the checked heads the
-oracle's fp32 scores go to the GPU selection (bit-exact index sets required) and the oracle's
-index sets go to the GPU mask builder and attention; 4,096 seeded (token, head) rows of the
-checked heads plus the first and last row of every prefill chunk are compared with the
+Checked heads: one Q head in every KV group (4 at the 7B shape, 8 at the 14B shape), at a
+position in the group that moves from the first head of the first group to the last head
+of the last. For each workload: the GPU runs every prefill chunk stage by stage; for the
+checked heads the oracle's fp32 scores go to the GPU selection (bit-exact index sets
+required) and the oracle's index sets go to the GPU mask builder, whose block-mask bits,
+residual vertical lists and per-pattern counts must equal the oracle's computed blocks and
+residual verticals bit for bit on every query block of every prefill chunk; the attended
+pairs counted from those counts (the benchmark's FLOP count) must equal the sum of |A(i)|
+over every row, taken from the oracle's blocks. 4,096 seeded (token, head) rows spread over
+the checked heads, plus the first and last row of every prefill chunk, are compared with the
 oracle (max-abs 2e-2, mean-relative 1e-3). The product entry point q1m_dca_sparse_prefill
 (the benchmark's call) is run on the same inputs: it ranks the GPU's own fp32 scores, so at a
 near-tie it may keep another index than the fp64 oracle. Its selection is therefore checked
@@ -14,12 +20,14 @@ unchecked head must match the stage-by-stage GPU run at the parity tolerance (bi
 in deterministic mode).
 """
 import os
+import time
 
 import numpy as np
 import pytest
 import torch
 
 from long_context_prefill_dca_b200 import q1m
+from long_context_prefill_dca_b200.accounting import pairs_from_counts
 from long_context_prefill_dca_b200.layer import Layer, Stages
 from oracle import dca_vs as O
 from synth import configs as C
@@ -33,8 +41,62 @@ WORKLOADS = [C.L7B_128K, C.L14B_256K, C.L7B_1M, C.L14B_1M]
 
 
 def checked_heads(w):
-    # one Q head in the first and one in the last KV group
-    return [0, w.n_q_heads - 1]
+    """One Q head per KV group: head g G + floor(g (G - 1) / (Hkv - 1)) of group g, so the
+    first head of the first group and the last head of the last are both checked."""
+    G, hkv = w.group, w.n_kv_heads
+    if hkv == 1:
+        return [0]
+    return [g * G + (g * (G - 1)) // (hkv - 1) for g in range(hkv)]
+
+
+def unpack_bits(words, nkb):
+    m = np.asarray(words).astype(np.uint32)
+    bits = (m[..., None] >> np.arange(32, dtype=np.uint32)) & 1
+    return bits.reshape(*m.shape[:-1], -1)[..., :nkb].astype(bool)
+
+
+def check_chunk_masks(w, orc, sel, heads, mask, resid, cnt):
+    """GPU masks, residual lists and counts of one prefill chunk against the oracle's
+    computed blocks and residual verticals for `heads`, bit for bit. Returns the oracle's
+    attended pairs of those heads, sum over rows i of |A(i)|, counted row by row from its
+    blocks and vertical columns."""
+    s0, e = sel.s0, sel.e
+    nkb, nqb = (e + 127) // 128, (e - s0 + 127) // 128
+    Lb = O.dca_len(w) // 128
+    idx = torch.tensor(heads, device=mask.device)
+    bits = unpack_bits(mask.index_select(0, idx).cpu().numpy(), nkb)
+    rs = resid.index_select(0, idx).cpu().numpy() if resid.shape[-1] else None
+    cn = cnt.index_select(0, idx).cpu().numpy()
+    kseg = np.arange(nkb) // Lb
+    pairs = 0
+    for k, h in enumerate(heads):
+        Vh = np.asarray(sel.V[h])
+        for qb in range(nqb):
+            b = s0 // 128 + qb
+            ref = orc.blocks(h, b, sel)
+            assert np.array_equal(bits[k, qb], ref), (w.name, s0, h, qb)
+            rv = O.residual_verticals(Vh, ref, b, e)
+            c = cn[k, qb]
+            assert c[6] == len(rv) and c[7] == 0, (w.name, s0, h, qb)
+            if len(rv):
+                assert np.array_equal(rs[k, qb, :len(rv)], rv), (w.name, s0, h, qb)
+            cb = b // Lb
+            seg = np.where(kseg == cb, 0, np.where(kseg == cb - 1, 1, 2))
+            assert [int(np.sum(ref & (seg == x))) for x in range(3)] == list(c[:3]), (s0, h, qb)
+            rseg = rv // O.dca_len(w)
+            assert [int(np.sum(rseg == cb)), int(np.sum(rseg == cb - 1)),
+                    int(np.sum(rseg <= cb - 2))] == list(c[3:6]), (s0, h, qb)
+            # |A(i)| for every row i of the block: full computed blocks below it, the causal
+            # part of its own block if computed, and the vertical columns j <= i outside them
+            r0, r1 = 128 * b, min(128 * b + 127, e - 1)
+            i = np.arange(r0, r1 + 1)
+            below = 128 * int(np.sum(ref[:b]))
+            own = (i - r0 + 1) if ref[b] else 0
+            extra = np.searchsorted(np.sort(rv), i, side="right")
+            pairs += int(np.sum(below + own + extra))
+    gpu_pairs = pairs_from_counts(cn, s0, e)
+    assert gpu_pairs == pairs, (w.name, s0, gpu_pairs, pairs)
+    return pairs
 
 
 def sampled_rows(w):
@@ -79,6 +141,9 @@ def test_full_size_sampled_rows(w):
     orc = O.Oracle(x["q"], x["k"], x["v"], w)
     rows = sampled_rows(w)
     heads = sorted(rows)
+    assert heads == checked_heads(w)
+    t_orc = 0.0                         # seconds spent in the oracle
+    n_pairs = 0
     st = Stages(w)
     out = torch.full((w.seq_len, w.n_q_heads, w.head_dim), float("nan"), device=dev)
     ref_rows = {h: [] for h in heads}
@@ -87,7 +152,9 @@ def test_full_size_sampled_rows(w):
     spare = 1                           # an unchecked head: product ~ stages
     assert spare not in heads
     for s0, e in O.prefill_chunks(w):
+        t0 = time.time()
         sel = orc.select_chunk(s0, e, heads)
+        t_orc += time.time() - t0
         st.keys(g["k"], g["v"], s0, e)
         st.queries(g["q"], s0, e)
         vert, slash = st.estimate(g["q"], s0, e)
@@ -113,6 +180,11 @@ def test_full_size_sampled_rows(w):
         for h in heads:
             assert np.array_equal(Vc[h], sel.V[h]) and np.array_equal(Sc[h], sel.S[h]), (w.name, s0, h)
         mask, resid, cnt = st.masks(V, S, s0, e)
+        torch.cuda.synchronize()
+        q1m.check_status()
+        t0 = time.time()
+        n_pairs += check_chunk_masks(w, orc, sel, heads, mask, resid, cnt)
+        t_orc += time.time() - t0
         st.attn(s0, e, mask, resid, cnt)
         st.merge(s0, e, out)
         torch.cuda.synchronize()
@@ -120,7 +192,9 @@ def test_full_size_sampled_rows(w):
         for h in heads:
             r = rows[h][(rows[h] >= s0) & (rows[h] < e)]
             if len(r):
+                t0 = time.time()
                 o, _ = orc.attend_rows(r, h, sel)
+                t_orc += time.time() - t0
                 ref_rows[h].append((r, o))
                 same = np.array_equal(own.V[h], sel.V[h]) and np.array_equal(own.S[h], sel.S[h])
                 n_swapped += not same
@@ -133,7 +207,9 @@ def test_full_size_sampled_rows(w):
             ref_all.append(o)
     got, ref = np.concatenate(got_all), np.concatenate(ref_all)
     err = np.abs(got - ref)
-    print(f"{w.name}: {len(got)} rows, oracle-fed max-abs {err.max():.2e} mean-rel {rel(got, ref):.2e}")
+    print(f"{w.name}: heads {heads}, masks bit-exact on every chunk, {n_pairs:.0f} attended "
+          f"pairs; {len(got)} rows, oracle-fed max-abs {err.max():.2e} mean-rel "
+          f"{rel(got, ref):.2e}; oracle {t_orc:.0f} s")
     assert np.all(np.isfinite(got))
     assert err.max() <= MAX_ABS and rel(got, ref) <= MEAN_REL
     stage_spare = out[:, spare].clone()
