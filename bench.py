@@ -34,7 +34,17 @@ UNIT = "TFLOP/s"
 
 
 KERNEL_SOURCES = ("attn_tc.cuh", "q1m_device.cuh", "exp2_poly.h")
-TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "block_sparse_attn_dram_7b-1m.md")
+
+# DRAM traffic of one attention launch, from a one-launch ncu capture of a small case
+# (dram__bytes_read.sum + dram__bytes_write.sum), with the sha256 of the kernel's sources at
+# capture time: the figure is reported only while the sources still hash to it. The capture
+# is the 7B-shape 131,072-token workload's last prefill chunk; the 1M-token layer is not
+# captured (its launches run for seconds with tens of GB resident), so its traffic is null.
+SMALL_CASE_TRAFFIC = {
+    "workload": "7b-128k", "chunk": 3,
+    "bytes_per_launch": None,
+    "kernel_source_sha256": None,
+}
 
 
 def kernel_source_hash() -> str:
@@ -50,20 +60,13 @@ def kernel_source_hash() -> str:
     return hashlib.sha256(text.encode()).hexdigest()
 
 
-def kernel_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu summary of the 7B@1M layer, or
-    None when the workload differs or the kernel's code changed since the capture (the hash
-    of its sources is recorded beside the figure)."""
-    if workload != "7b-1m" or not os.path.exists(TRAFFIC_PROFILE):
+def small_case_traffic():
+    """The small case's DRAM bytes per attention launch while the kernel is unchanged since
+    its capture, else None."""
+    t = SMALL_CASE_TRAFFIC
+    if t["bytes_per_launch"] is None or t["kernel_source_sha256"] != kernel_source_hash():
         return None
-    rec = {}
-    for line in open(TRAFFIC_PROFILE):
-        if ":" in line and line.split(":", 1)[0] in ("traffic_per_launch_bytes", "kernel_source_sha256"):
-            k, v = line.split(":", 1)
-            rec[k] = v.strip()
-    if rec.get("kernel_source_sha256") != kernel_source_hash() or "traffic_per_launch_bytes" not in rec:
-        return None
-    return float(rec["traffic_per_launch_bytes"])
+    return t["bytes_per_launch"]
 
 
 def parse():
@@ -205,47 +208,80 @@ def blas_threads() -> int:
         return 1
 
 
-def oracle_sample(w, x, dense_pairs_total, n_rows=4):
-    """Time the fp64 oracle on a bounded sample of the layer and extrapolate to the whole
-    layer. Returns (seconds per layer, description, total pairs estimate)."""
+FULL_ORACLE_ROWS = 1 << 14    # rows x heads up to which the oracle runs the whole layer
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, x, dense_pairs_total, n_heads=4, rows_per_head=16, orc=None, t_krot=None):
+    """Time the fp64 oracle, as it stands, on a bounded sample of the layer and extrapolate to
+    the whole layer. The sample: the key rotation of the last KV group, the estimator and
+    selection of the last prefill chunk for `n_heads` Q heads of that group, and the attention
+    of the last `rows_per_head` rows of each of those heads. The layer estimate scales the
+    attention time by attended pairs (the sampled heads' block density applied to every row),
+    the estimator time by estimator rows x keys over all chunks, and the rotation by KV heads.
+    `orc` / `t_krot` reuse an oracle whose rotated keys are already computed and the time that
+    took (the reference arm's later steps). Returns a dict."""
     import numpy as np
     from oracle import dca_vs as O
-    orc = O.Oracle(x["q"], x["k"], x["v"], w)
-    h = w.n_q_heads - 1
-    g = h // w.group
+    if w.seq_len * w.n_q_heads <= FULL_ORACLE_ROWS:
+        # small enough for the whole layer: no extrapolation
+        t0 = time.perf_counter()
+        O.Oracle(x["q"], x["k"], x["v"], w).run()
+        t = time.perf_counter() - t0
+        return {"t_layer": t, "sample_s": t, "pairs_total": dense_pairs_total if w.dense else None,
+                "desc": f"fp64 oracle (numpy), the whole layer: every row of every head ({t:.1f} s)",
+                "orc": None, "t_krot": None, "extrapolated": False}
+    g = w.n_kv_heads - 1
+    heads = [g * w.group + i for i in range(min(n_heads, w.group))]
+    sample_t0 = time.perf_counter()
+    if orc is None:
+        orc = O.Oracle(x["q"], x["k"], x["v"], w)
+    if t_krot is None:
+        t0 = time.perf_counter()
+        orc.krot(g)
+        t_krot = time.perf_counter() - t0
     chunks = list(O.prefill_chunks(w))
     s0, e = chunks[-1]
-    t0 = time.perf_counter()
-    orc.krot(g)
-    t_krot = time.perf_counter() - t0
     t_est, density = 0.0, 1.0
     sel = O.ChunkSelection(s0, e)
     if not w.dense:
         R = O.estimator_rows(s0, e, w)
-        t0 = time.perf_counter()
-        vt, sl, _ = O.estimate_head(orc.q_rows(R, h), R, orc.krot(g), e, w)
-        V, S = O.select_head(vt, sl, w)
-        t_est = time.perf_counter() - t0
         sel.V = [None] * w.n_q_heads
         sel.S = [None] * w.n_q_heads
-        sel.V[h], sel.S[h] = V, S
+        dens = []
+        t0 = time.perf_counter()
+        for h in heads:
+            vt, sl, _ = O.estimate_head(orc.q_rows(R, h), R, orc.krot(g), e, w)
+            sel.V[h], sel.S[h] = O.select_head(vt, sl, w)
+        t_est = time.perf_counter() - t0
         nb = (e + 127) // 128
-        dens = [O.computed_blocks(S, b, e)[: b + 1].mean() for b in range(s0 // 128, nb, 64)]
+        for h in heads:
+            dens += [O.computed_blocks(sel.S[h], b, e)[: b + 1].mean() for b in range(s0 // 128, nb, 64)]
         density = float(np.mean(dens))
-    rows = np.arange(e - n_rows, e)
+    rows = np.arange(e - rows_per_head, e)
     t0 = time.perf_counter()
-    orc.attend_rows(rows, h, sel)
+    for h in heads:
+        orc.attend_rows(rows, h, sel)
     t_att = time.perf_counter() - t0
-    pairs_sample = float(sum(int(orc.attended(int(i), h, sel).sum()) for i in rows))
+    sample_s = time.perf_counter() - sample_t0
+    pairs_sample = float(sum(int(orc.attended(int(i), h, sel).sum()) for h in heads for i in rows))
     pairs_total = dense_pairs_total * density
     est_rows_keys = sum(w.n_q_heads * ee for _, ee in chunks)
-    t_layer = (t_att / pairs_sample * pairs_total + t_est / e * est_rows_keys +
+    t_layer = (t_att / pairs_sample * pairs_total + t_est / (len(heads) * e) * est_rows_keys +
                t_krot * w.n_kv_heads)
-    desc = (f"fp64 oracle, head {h}: key rotation of 1 KV head ({t_krot:.1f}s), estimator of "
-            f"the last chunk ({t_est:.1f}s), attention of the last {n_rows} rows "
-            f"({t_att:.1f}s, {pairs_sample:.3g} pairs); extrapolated to the layer by pairs "
-            f"(density {density:.3f}), estimator rows x keys and KV heads")
-    return t_layer, desc, pairs_total
+    desc = (f"fp64 oracle (numpy; BLAS matmuls threaded, the rest on one core), KV group {g}: key "
+            f"rotation ({t_krot:.1f} s), estimator + selection of the last prefill chunk for Q "
+            f"heads {heads} ({t_est:.1f} s), attention of the last {rows_per_head} rows of each "
+            f"({t_att:.1f} s, {pairs_sample:.3g} pairs); extrapolated to the layer by attended "
+            f"pairs (block density {density:.3f}), estimator rows x keys and KV heads")
+    return {"t_layer": t_layer, "sample_s": sample_s, "desc": desc, "pairs_total": pairs_total,
+            "orc": orc, "t_krot": t_krot, "pairs_sample": pairs_sample, "extrapolated": True}
 
 
 def estimator_work(w) -> dict:
@@ -291,33 +327,78 @@ def dense_pairs(w) -> float:
     return n * (n + 1) / 2 * w.n_q_heads
 
 
+L2_FLUSH_BYTES = 512 << 20    # written between timed steps when the inputs are smaller
+
+
+def config_of(w, args, world=1, w_full=None, sharded=False) -> dict:
+    """The workload description both arms print."""
+    from long_context_prefill_dca_b200 import q1m
+    w_full = w_full or w
+    in_bytes = (w.seq_len * (w.n_q_heads + 2 * w.n_kv_heads) * w.head_dim *
+                (2 if w.in_dtype == "bf16" else 4))
+    return {"workload": w.name, "seq_len": w.seq_len, "n_q_heads": w_full.n_q_heads,
+            "n_kv_heads": w_full.n_kv_heads, "head_dim": w.head_dim,
+            "heads_per_rank": [w.n_q_heads, w.n_kv_heads],
+            "dca_chunk": w.dca_chunk, "local_window": w.local_window,
+            "yarn_s": w.yarn_s, "prefill_chunk": w.prefill_chunk,
+            "chunking": (f"equal-cost x{w.equal_cost_chunks}" if w.equal_cost_chunks else "fixed"),
+            "prefill_chunks": [list(b) for b in q1m.prefill_bounds(w)],
+            "vs_budget": [w.vs_vertical, w.vs_slash], "inputs": w.in_dtype,
+            "mma": "f16 x f16 -> f32 (rotated, scaled Q and K beyond +-65,504 are refused "
+                   "with Q1M_ERR_RANGE)",
+            "out": args.out_dtype,
+            "parallelism": (f"KV-head groups split over {world} GPUs" if sharded else
+                            f"replicas x{world}" if world > 1 else "single GPU"),
+            "l2": (f"inputs ({in_bytes / 1e9:.2f} GB) larger than L2 (126 MB); no flush"
+                   if in_bytes >= L2_FLUSH_BYTES else
+                   f"inputs ({in_bytes / 1e6:.1f} MB) within L2: a {L2_FLUSH_BYTES >> 20} MiB "
+                   "buffer is written between timed steps, each step timed on its own")}
+
+
 def run_reference(args):
-    """The reference arm: the oracle as it stands on the host cores, bounded samples."""
+    """The reference arm: the oracle as it stands on the host cores. Each step times one
+    bounded sample of the workload (the first step also rotates the sampled KV group's keys,
+    which later steps reuse); value is the layer's attention FLOPs over the layer time
+    extrapolated from that sample."""
     from synth import configs as C
     from synth import inputs as I
-    w = C.BY_NAME[args.workload].with_(equal_cost_chunks=args.equal_cost_chunks)
+    w = C.BY_NAME[args.workload].with_(equal_cost_chunks=args.equal_cost_chunks,
+                                        out_dtype=args.out_dtype)
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     x = I.generate(w)
     dp = dense_pairs(w)
-    times = []
-    desc, pairs = "", dp
+    layer_s, sample_s = [], []
+    orc, t_krot, res = None, None, None
     for it in range(args.warmup + args.steps):
-        t_layer, desc, pairs = oracle_sample(w, x, dp)
+        res = oracle_sample(w, x, dp, n_heads=1, rows_per_head=4, orc=orc, t_krot=t_krot)
+        orc, t_krot = res["orc"], res["t_krot"]
         if it >= args.warmup:
-            times.append(t_layer)
-    t = sum(times) / len(times)
-    flops = 4.0 * w.head_dim * pairs
+            layer_s.append(res["t_layer"])
+            sample_s.append(res["sample_s"])
+    t = sum(layer_s) / len(layer_s)
+    if res["pairs_total"] is None:   # the whole sparse layer ran: count its attended pairs
+        from oracle import dca_vs as O
+        orc = O.Oracle(x["q"], x["k"], x["v"], w)
+        res["pairs_total"] = float(sum(int(orc.attended(i, h, sel).sum())
+                                       for sel in (orc.select_chunk(a, b) for a, b in O.prefill_chunks(w))
+                                       for h in range(w.n_q_heads) for i in range(sel.s0, sel.e)))
+    flops = 4.0 * w.head_dim * res["pairs_total"]
     value = flops / t / 1e12
     line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": sum(sample_s) / len(sample_s) * 1e3,
+            "ms_per_layer_extrapolated": t * 1e3 if res["extrapolated"] else None,
+            "extrapolated": res["extrapolated"],
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) + planted sinks/bands)",
-            "config": {"workload": w.name, "seq_len": w.seq_len, "n_q_heads": w.n_q_heads,
-                       "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim},
+            "config": config_of(w, args),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
-                             "kind": "oracle", "sample": desc},
+                             "host_cores": host_cores(), "kind": "oracle",
+                             "extrapolated": res["extrapolated"],
+                             "sample_seconds": sum(sample_s) / len(sample_s),
+                             "sample": res["desc"] + "; ms_per_step is one sample's measured time"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -365,6 +446,8 @@ def main():
                       dtype=torch.bfloat16 if args.out_dtype == "bf16" else torch.float32,
                       device=device)
     stream = torch.cuda.current_stream(device)
+    in_bytes = sum(t.numel() * t.element_size() for t in g.values())
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device) if in_bytes < L2_FLUSH_BYTES else None
 
     def step():
         layer(g["q"], g["k"], g["v"], out=out, stream=stream)
@@ -387,12 +470,27 @@ def main():
     torch.cuda.synchronize(device)
     q1m.profile_enable(True)
     n0 = q1m.launch_count()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    torch.cuda.synchronize(device)
+    if flush is None:
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(device)
+        ms_total = ev0.elapsed_time(ev1)
+    else:
+        # inputs that fit in L2: each step is timed on its own, after a write of a buffer
+        # larger than L2 that evicts the previous step's data
+        evs = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step()
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize(device)
+        ms_total = sum(a.elapsed_time(b) for a, b in evs)
     if world > 1:
         dist.barrier()
     launches = q1m.launch_count() - n0
@@ -400,7 +498,7 @@ def main():
     q1m.profile_enable(False)
     clk = clocks.stop()
     q1m.check_status(stream)
-    ms_step = max_over_ranks(ev0.elapsed_time(ev1), world, device) / args.steps
+    ms_step = max_over_ranks(ms_total, world, device) / args.steps
     job_flops = sum_over_ranks(flops, world, device)   # replicas: world x flops
     value = job_flops / (ms_step * 1e-3) / 1e12
     allgather_ms = None
@@ -446,10 +544,16 @@ def main():
     # per launch: the timed region's attention FLOPs over its attention-kernel launches,
     # divided by the average launch duration (events on the launching stream)
     achieved = (flops * args.steps / attn_n) / (attn_ms / attn_n * 1e-3) / 1e12 if attn_n else None
-    roofline = {"bound": "tensor", "kernel": "block_sparse_attn_kernel<128>",
+    t_small = small_case_traffic()
+    roofline = {"bound": "tensor", "kernel": f"block_sparse_attn_kernel<{w.head_dim}>",
                 "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
-                "frac": achieved / sustained if achieved else None, "traffic": kernel_traffic(w.name),
-                "traffic_unit": "DRAM bytes per launch (ncu, profiles/block_sparse_attn_dram_7b-1m.md)",
+                "frac": achieved / sustained if achieved else None,
+                "traffic": t_small if w.name == SMALL_CASE_TRAFFIC["workload"] else None,
+                "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + "
+                                "dram__bytes_write.sum, one launch of the small case)",
+                "traffic_small_case": {"workload": SMALL_CASE_TRAFFIC["workload"],
+                                       "prefill_chunk": SMALL_CASE_TRAFFIC["chunk"],
+                                       "bytes_per_launch": t_small},
                 "peak_source": f"{src} bf16 sustained (MEASURED_PEAKS.json); fp16 operands run at the bf16 rate",
                 "frac_of_burst": achieved / burst if achieved else None,
                 "layer_frac": value / world / sustained}
@@ -469,29 +573,18 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t_layer, desc, cpu_pairs = oracle_sample(w, x, dense_pairs(w))
-        cpu = {"value": 4.0 * w.head_dim * pairs / t_layer / 1e12, "unit": UNIT,
-               "cores": blas_threads(), "kind": "oracle", "sample": desc,
-               "seconds_per_layer_extrapolated": t_layer}
+        res = oracle_sample(w, x, dense_pairs(w))
+        cpu = {"value": 4.0 * w.head_dim * pairs / res["t_layer"] / 1e12, "unit": UNIT,
+               "cores": blas_threads(), "host_cores": host_cores(), "kind": "oracle",
+               "extrapolated": res["extrapolated"], "sample_seconds": res["sample_s"],
+               "sample": res["desc"], "seconds_per_layer": res["t_layer"]}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
             "dtype": "f16", "data": "synthetic (seeded N(0,1) + planted sinks/bands, bf16)",
-            "config": {"workload": w.name, "seq_len": w.seq_len, "n_q_heads": w_full.n_q_heads,
-                       "n_kv_heads": w_full.n_kv_heads, "head_dim": w.head_dim,
-                       "heads_per_rank": [w.n_q_heads, w.n_kv_heads],
-                       "dca_chunk": w.dca_chunk, "local_window": w.local_window,
-                       "yarn_s": w.yarn_s, "prefill_chunk": w.prefill_chunk,
-                       "chunking": (f"equal-cost x{w.equal_cost_chunks}" if w.equal_cost_chunks
-                                    else "fixed"),
-                       "prefill_chunks": [list(b) for b in q1m.prefill_bounds(w)],
-                       "vs_budget": [w.vs_vertical, w.vs_slash], "inputs": "bf16",
-                       "mma": "f16 x f16 -> f32", "out": args.out_dtype,
-                       "parallelism": (f"KV-head groups split over {world} GPUs" if sharded else
-                                       f"replicas x{world}" if world > 1 else "single GPU"),
+            "config": {**config_of(w, args, world, w_full, sharded),
                        "allgather_ms": allgather_ms,
-                       "l2": "inputs (9.6 GB) far larger than L2 (126 MB); no flush",
                        "attended_pairs": job_flops / (4.0 * w.head_dim), "block_density": density,
                        "ms_per_layer": ms_step},
             "roofline": roofline, "estimator": estimator, "stages": stages,

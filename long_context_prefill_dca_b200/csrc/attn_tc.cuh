@@ -15,9 +15,10 @@
 //    block right after slot 0, so in dense mode the lists coincide and in sparse mode
 //    (Toeplitz block masks) they mostly do.
 //  * Each item walks its key blocks from a start taken from a global count of the tiles all
-//    CTAs have issued (wrapping around its range), so CTAs that stream the same K/V range
-//    stay at about the same tile and share it in L2 (see g_k3_cursor); deterministic mode
-//    starts every walk at its first block.
+//    CTAs have issued (wrapping around its range; for intra items the count is first taken
+//    modulo the DCA chunk's block count), so CTAs that stream the same K/V range stay at
+//    about the same tile and share it in L2 (see g_k3_cursor); deterministic mode starts
+//    every walk at its first block.
 //  * Warp roles: warps 0-3 softmax of slot 0, warps 4-7 softmax of slot 1, warp 8 loads
 //    (TMA for key blocks, cp.async gathers for residual vertical columns), warp 9 issues
 //    tcgen05.mma and owns tensor memory, warp 10 loads V tiles, warp 11 idles; the softmax
@@ -285,7 +286,12 @@ __device__ void k3_producer(K3Smem<D>& sm, const K3Args& a, const CUtensorMap* m
           unsigned long long c = 0;
           if (leader) c = *(volatile unsigned long long*)&g_k3_cursor;
           c = __shfl_sync(0xFFFFFFFFu, c, 0);
-          start = lo + (int)((c / gridDim.x) % (unsigned long long)(hi - lo + 1));
+          // intra items' ranges share lo but differ in length: taking the clock modulo the
+          // DCA chunk's block count first puts every intra item whose range reaches that
+          // phase on the same block
+          unsigned long long ph = c / gridDim.x;
+          if (I.x == 0) ph %= (unsigned long long)(a.L / 128);
+          start = lo + (int)(ph % (unsigned long long)(hi - lo + 1));
         }
         if (ok) {
           if (leader) { sm.walk_start[slot] = start; mbar_arrive(&sm.start_full[slot]); }
