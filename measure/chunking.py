@@ -1,7 +1,7 @@
 """Per-chunk timing of the chunked prefill with fixed-size chunks and with equal-cost chunks
 (the pages' sizing of chunks by attention cost, here on one GPU).
 
-    python -m long_context_prefill_dca_b200.chunking --workload 7b-1m --chunks 8
+    python -m measure.chunking --workload 7b-1m --chunks 8
 
 For each mode, runs every prefill chunk through the stage kernels (the same ones the layer
 runs) on the seeded synthetic inputs, times each chunk and its attention kernel with CUDA

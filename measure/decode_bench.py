@@ -1,6 +1,6 @@
 """Timing of one DCA decode step (q1m_dca_decode) at long context on the seeded inputs.
 
-    python -m long_context_prefill_dca_b200.decode_bench --workload 7b-1m --steps 20
+    python -m measure.decode_bench --workload 7b-1m --steps 20
 
 Builds the fp16 cache of the first n - 1 tokens with the prefill's key rotation, then times
 the decode step of the token at n - 1 (append, query views, decode kernel, merge) for a few

@@ -2,7 +2,7 @@
 sweeps (the measurement behind the pages' sparsity refinement: keep the sparse config's
 accuracy loss small).
 
-    python -m long_context_prefill_dca_b200.recall --workload small-sparse [--sweep 0.5,1,2]
+    python -m measure.recall --workload small-sparse [--sweep 0.5,1,2]
 
 Runs the layer twice through the C ABI, sparse and dense, and reports
 recall_i = exp(lse_sparse_i - lse_dense_i) (q1m_attention_recall): the share of each row's

@@ -16,7 +16,7 @@ Sources (page title, section):
   [P5]  "Qwen2.5-1M リリース" (agentlenshq), "Sparse Attention" (chunked prefill, chunk
         32,768) and "Deploy Qwen2.5-1M Models Locally" (chunk 131,072 via
         --max-num-batched-tokens).
-Readings where the pages leave a step open are marked READING and listed in the design doc.
+Readings where the pages leave a step open are marked READING.
 
 Every function here is pinned by tests in tests/test_oracle_pins.py.
 """
