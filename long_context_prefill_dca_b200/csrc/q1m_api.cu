@@ -234,7 +234,9 @@ EstLayout est_layout(int64_t e, int hq, int hkv, int d) {
   L.n_mt = (G * 64 + 127) / 128;
   L.m_pad = L.n_mt * 128;
   L.nkt = (int)((e + 127) / 128);
-  int ns = (296 + hkv * L.n_mt - 1) / (hkv * L.n_mt);
+  // pass A runs two CTAs per SM: split the key range so every CTA is resident in one wave
+  // of 2 x 148
+  int ns = 296 / (hkv * L.n_mt);
   L.nsplit = ns < 1 ? 1 : (ns > L.nkt ? L.nkt : ns);
   size_t off = 0;
   L.est_q = off; off = align_up(off + (size_t)4 * hkv * L.m_pad * d * 2);
@@ -472,7 +474,7 @@ q1m_status run_estimate_d(const void* q, const uint16_t* k_rot, int64_t ld_token
     const int grid = (int)(W < dev.sms ? W : dev.sms);
     est_pass_b_kernel<D><<<grid, EB_THREADS, smem, st>>>(m_est64, m_k, a);
     Q1M_LAUNCHED();
-    est_slash_reduce_kernel<<<blocks_for((int64_t)hq * e, 256), 256, 0, st>>>(a, slash);
+    est_slash_reduce_kernel<<<dim3(blocks_for(e, 256), hq), 256, 0, st>>>(a, slash);
     Q1M_LAUNCHED();
   }
   return Q1M_OK;

@@ -97,10 +97,44 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// try_wait with a suspend-time hint: the thread may be suspended until the phase completes
+// (or hint_ns nanoseconds pass) instead of returning at once, so a warp that waits for
+// long takes no issue slots from the warps that work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait whose tries suspend the thread (up to 20 us each) until the phase completes.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long budget = g_wait_cycles;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (failed()) return false;
+    if ((unsigned long long)(clock64() - t0) > budget) {
+      latch(Q1M_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // The same wait taken by a whole warp: the outcome is agreed by all 32 lanes, so a wait
 // that runs out in one lane never leaves the others at a warp-synchronous instruction.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity));
+}
+
+__device__ __forceinline__ bool mbar_wait_sleep_warp(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait_sleep(bar, parity));
 }
 
 // Named barrier over `count` threads that also ANDs a predicate across them.
@@ -264,6 +298,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
       "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
       : Q1M_R8(0), Q1M_R8(8), Q1M_R8(16), Q1M_R8(24)
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : Q1M_R8(0)
       : "r"(taddr)
       : "memory");
 }

@@ -11,11 +11,16 @@
 // by its DCA chunk class (see est_queries_kernel).
 //  pass A: rows as M (128 rows per tile), keys as N; online max/sum per row over a range of
 //          key tiles; partial (max, sum) per split, merged into the row's log2-sum-exp2.
-//  pass B: keys as M (128 keys per tile), est rows as N (<= 448 TMEM columns). Each thread
-//          owns one key: its vertical score is a thread-local sum over rows. Slash sums go
-//          through shared memory along diagonals (192 offsets per key tile, written per tile
-//          and summed over the two tiles that touch each offset in a fixed order), so the
-//          scores are deterministic.
+//  pass B: keys as M (128 keys per tile), est rows as N (<= 448 TMEM columns, in two
+//          accumulators: heads 0..3 and heads 4..6, so the MMA of one overlaps the epilogue
+//          of the other). One epilogue warp per (pair of heads, 32-key quarter), the two
+//          heads' values packed in float2 so that every add, shared-memory access and
+//          exponential argument serves both; each thread owns one key, so its vertical
+//          scores are thread-local sums over rows. Slash sums are sums along diagonals: each
+//          warp transposes its 32 keys x 8 rows of p through its own shared-memory buffer
+//          and sums the 39 diagonals they touch; the four quarters' diagonal partials are
+//          added per tile (192 offsets) and the two tiles that touch each offset are summed
+//          later, always in the same order, so the scores are deterministic.
 #pragma once
 
 #include "q1m_device.cuh"
@@ -24,12 +29,14 @@ namespace q1m {
 
 constexpr int EA_THREADS = 192;   // warps 0-3 softmax, 4 loader, 5 MMA
 constexpr int EA_NK = 2;
-constexpr int EB_THREADS = 576;   // warps 0-15 epilogue (4 groups), 16 loader, 17 MMA
-constexpr int EB_GROUPS = 4;      // epilogue groups of 4 warps (one per TMEM lane quarter)
-constexpr int EB_STEP = 16;       // est rows per epilogue step
-constexpr int EB_NK = 2;
+constexpr int EB_PAIRS = 4;                            // head pairs (0,1) (2,3) (4,5) (6)
+constexpr int EB_THREADS = 32 * (4 * EB_PAIRS + 2);    // warps 0-15 epilogue, 16 loader, 17 MMA
+constexpr int EB_STEP = 8;        // est rows per epilogue step
+constexpr int EB_PITCH = EB_STEP + 1;   // float2 per key in a warp's transpose buffer (no bank conflicts)
+constexpr int EB_ACC0_HEADS = 4;  // accumulator 0 holds heads 0..3, accumulator 1 heads 4..6
 constexpr int EB_MAX_ROWS = 448;
 constexpr int EB_U = 192;         // offsets per key tile (64 + 128 - 1 used)
+constexpr int EB_DQ = 96;         // diagonal partials of one key quarter (32 + 64 - 1 used)
 
 struct EstArgs {
   int64_t r_lo, e;     // estimator rows [r_lo, e)
@@ -51,6 +58,44 @@ __device__ __forceinline__ int est_class(const EstArgs& a, int kt) {
   const int64_t kc = (int64_t)kt * 128 / a.L;
   const int64_t d = a.c_hi - kc;
   return d >= 3 ? 3 : (int)d;
+}
+
+// One key tile of a pass A row: the online log2-sum-exp2 (mx, l) of row values x[0..127]
+// (log2-scaled logits). MASKED: keys c > lim are not causal for the row.
+template <bool MASKED>
+__device__ __forceinline__ void est_a_tile(float (&x)[128], int64_t lim, float& mx, float& l) {
+  if (MASKED) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c) if (c > lim) x[c] = -INFINITY;
+  }
+  // tile maximum: eight independent chains, then a tree
+  float m8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m8[k] = x[k];
+#pragma unroll
+  for (int c = 8; c < 128; c += 8)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], x[c + k]);
+#pragma unroll
+  for (int wdt = 4; wdt >= 1; wdt /= 2)
+#pragma unroll
+    for (int k = 0; k < wdt; ++k) m8[k] = fmaxf(m8[k], m8[k + wdt]);
+  const float mn = fmaxf(mx, m8[0]);
+  if (mn == -INFINITY) return;
+  // 2^(x - mn): packed subtractions, four independent packed sums
+  const uint64_t nmn = f2_pack(-mn, -mn);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int c = 0; c < 64; ++c) {
+    float d0, d1;
+    f2_unpack(f2_add(f2_pack(x[2 * c], x[2 * c + 1]), nmn), d0, d1);
+    acc[c & 3] = f2_add(acc[c & 3], f2_pack(ex2(d0), ex2(d1)));
+  }
+  float s0, s1, s2, s3;
+  f2_unpack(f2_add(acc[0], acc[1]), s0, s1);
+  f2_unpack(f2_add(acc[2], acc[3]), s2, s3);
+  l = l * ex2(mx - mn) + ((s0 + s1) + (s2 + s3));
+  mx = mn;
 }
 
 // --------------------------------------------------------------------------------------
@@ -97,7 +142,7 @@ est_pass_a_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
       for (int kt = t0, n = 0; kt < t1 && ok; ++kt, ++n) {
         const int cls = est_class(a, kt);
         if (cls != cls_cur) {
-          ok = mbar_wait(&sm.q_empty, (qn & 1) ^ 1);
+          ok = mbar_wait_sleep(&sm.q_empty, (qn & 1) ^ 1);
           if (!ok) break;
           mbar_expect_tx(&sm.q_full, TILE);
           const int y = (int)(((int64_t)cls * a.hkv + g) * a.m_pad + mt * 128);
@@ -106,7 +151,7 @@ est_pass_a_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
           cls_cur = cls;
         }
         const int st = n % EA_NK;
-        ok = mbar_wait(&sm.k_empty[st], ((n / EA_NK) & 1) ^ 1);
+        ok = mbar_wait_sleep(&sm.k_empty[st], ((n / EA_NK) & 1) ^ 1);
         if (!ok) break;
         mbar_expect_tx(&sm.k_full[st], TILE);
         const int y = (int)((int64_t)g * a.ld_tokens + (int64_t)kt * 128);
@@ -122,13 +167,13 @@ est_pass_a_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
       for (int kt = t0, n = 0; kt < t1 && ok; ++kt, ++n) {
         const int cls = est_class(a, kt);
         if (cls != cls_cur) {
-          ok = mbar_wait(&sm.q_full, qn & 1);
+          ok = mbar_wait_sleep(&sm.q_full, qn & 1);
           if (!ok) break;
           ++qn;
           cls_cur = cls;
         }
         const int st = n % EA_NK, b = n & 1;
-        ok = mbar_wait(&sm.k_full[st], (n / EA_NK) & 1) && mbar_wait(&sm.s_free[b], ((n >> 1) & 1) ^ 1);
+        ok = mbar_wait_sleep(&sm.k_full[st], (n / EA_NK) & 1) && mbar_wait_sleep(&sm.s_free[b], ((n >> 1) & 1) ^ 1);
         if (!ok) break;
         tc_fence_after();
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -141,7 +186,7 @@ est_pass_a_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         if (kt + 1 >= t1 || est_class(a, kt + 1) != cls) mma_commit(&sm.q_empty);
       }
       mma_commit(&sm.drain);
-      mbar_wait(&sm.drain, 0);
+      mbar_wait_sleep(&sm.drain, 0);
     }
   } else {
     // softmax: thread t owns est row m = mt * 128 + t
@@ -153,29 +198,26 @@ est_pass_a_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     const uint32_t lb = tb + ((32u * (warp_id() & 3u)) << 16);
     float mx = -INFINITY, l = 0.f;
     bool ok = true;
+    // a warp whose 32 est rows are all padding (past the group's G x 64 rows) only frees the
+    // accumulator buffers
+    const bool warp_live = (mt * 128 + 32 * (int)(warp_id() & 3u)) / 64 < a.G;
     for (int kt = t0, n = 0; kt < t1 && ok; ++kt, ++n) {
       const int b = n & 1;
-      ok = mbar_wait_warp(&sm.s_full[b], (n >> 1) & 1);
+      ok = mbar_wait_sleep_warp(&sm.s_full[b], (n >> 1) & 1);
       if (!ok) break;
       tc_fence_after();
+      if (!warp_live) {
+        tc_fence_before();
+        mbar_arrive(&sm.s_free[b]);
+        continue;
+      }
       float x[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(lb + 128u * b + 32u * c, reinterpret_cast<uint32_t*>(x) + 32 * c);
       tc_fence_before();
       mbar_arrive(&sm.s_free[b]);
-      const int64_t lim = i - (int64_t)kt * 128;   // keys c <= lim are causal
-#pragma unroll
-      for (int c = 0; c < 128; ++c) if (c > lim) x[c] = -INFINITY;
-      float tmax = x[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) tmax = fmaxf(tmax, x[c]);
-      const float mn = fmaxf(mx, tmax);
-      if (mn == -INFINITY) continue;
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) sum += ex2(x[c] - mn);
-      l = l * ex2(mx - mn) + sum;
-      mx = mn;
+      if ((int64_t)kt * 128 + 127 > a.r_lo) est_a_tile<true>(x, i - (int64_t)kt * 128, mx, l);
+      else est_a_tile<false>(x, 0, mx, l);
     }
     if (ok) a.part[((int64_t)g * a.n_mt * 128 + m) * a.nsplit + split] = make_float2(live ? mx : -INFINITY, live ? l : 0.f);
   }
@@ -212,12 +254,182 @@ struct EBSmem {
   static constexpr int TILE = 128 * D * 2;
   static constexpr int EST = EB_MAX_ROWS * D * 2;
   alignas(1024) uint8_t est[EST];         // est rows, [half][row][64 halfs] swizzled
-  alignas(1024) uint8_t k[EB_NK][TILE];
-  float pbuf[EB_GROUPS][EB_STEP][128];    // per epilogue group: EB_STEP rows x 128 keys
-  float lse[EB_GROUPS][EB_MAX_ROWS];      // per epilogue group
-  uint64_t k_full[EB_NK], k_empty[EB_NK], e_full, e_empty, acc_full, acc_free, drain;
+  alignas(1024) uint8_t k[TILE];          // one key tile (the epilogue covers its reload)
+  float2 tbuf[4 * EB_PAIRS][32 * EB_PITCH];  // per epilogue warp: p of 32 keys x EB_STEP rows
+  float2 dsum[EB_PAIRS][4][EB_DQ];        // per head pair and key quarter: diagonal partials
+  float nlse[2 * EB_PAIRS][64];           // per head and est row: -(log2-sum-exp2)
+  uint64_t k_full, k_empty, e_full, e_empty, acc_full[2], acc_free[2], drain;
   uint32_t tmem_base;
 };
+
+// One element of a diagonal read: with q = (c <= l), load the packed pair at
+// (q ? ru : rd) + off and add it to da if q, else to db (predicated, no branch).
+template <int C, int OFF>
+__device__ __forceinline__ void diag_step(uint64_t& da, uint64_t& db, uint32_t ru, uint32_t rd, int l) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t.reg .b32 ad;\n\t.reg .b64 v;\n\t"
+      "setp.le.s32 q, %4, %5;\n\t"
+      "selp.b32 ad, %2, %3, q;\n\t"
+      "ld.shared.b64 v, [ad+%6];\n\t"
+      "@q add.rn.f32x2 %0, %0, v;\n\t"
+      "@!q add.rn.f32x2 %1, %1, v;\n\t}"
+      : "+l"(da), "+l"(db)
+      : "r"(ru), "r"(rd), "n"(C), "r"(l), "n"(OFF)
+      : "memory");
+}
+
+// One key tile of a pass B epilogue warp: p = 2^(s - lse) for the warp's 32 keys and its
+// head pair's 64 est rows, their vertical sums (returned packed (A, B)) and the diagonal
+// partials added into ds. MASKED: the tile reaches the estimator rows (keys after a row are
+// not causal) or the chunk has fewer than 64 rows.
+template <int D, bool TWO, bool MASKED>
+__device__ __forceinline__ uint64_t est_b_tile(EBSmem<D>& sm, const EstArgs& a, int pi, int hA, int half,
+                                               uint32_t lbA, float2* tw, float2* ds, uint32_t ru,
+                                               uint32_t rd, int l, int64_t j, int nR) {
+  uint64_t vs = 0ull;                                       // vertical sums (A, B)
+#pragma unroll 1
+  for (int s = 0; s < 64 / EB_STEP; ++s) {
+    uint32_t ra[EB_STEP], rb[EB_STEP];
+    tmem_ld8(lbA + (uint32_t)(s * EB_STEP), ra);
+    if (TWO) tmem_ld8(lbA + 64u + (uint32_t)(s * EB_STEP), rb);
+    if (s == 64 / EB_STEP - 1) {
+      // every TMEM read of this tile is done: the MMA may overwrite the accumulator
+      tc_fence_before();
+      __syncwarp();
+      if (l == 0) mbar_arrive(&sm.acc_free[half]);
+    }
+    // row pairs (c, c + 1) of one head are adjacent registers: packed adds on them, then
+    // each exponential's result is paired with the other head's for the transpose
+    const float4* nA4 = reinterpret_cast<const float4*>(&sm.nlse[hA][s * EB_STEP]);
+    const float4* nB4 = reinterpret_cast<const float4*>(&sm.nlse[hA + 1][s * EB_STEP]);
+    uint64_t pp[EB_STEP];
+#pragma unroll
+    for (int c4 = 0; c4 < EB_STEP / 4; ++c4) {
+      const float4 na = nA4[c4];
+      float dA[4], dB[4];
+      f2_unpack(f2_add(f2_pack(__uint_as_float(ra[4 * c4]), __uint_as_float(ra[4 * c4 + 1])), f2_pack(na.x, na.y)), dA[0], dA[1]);
+      f2_unpack(f2_add(f2_pack(__uint_as_float(ra[4 * c4 + 2]), __uint_as_float(ra[4 * c4 + 3])), f2_pack(na.z, na.w)), dA[2], dA[3]);
+      if (TWO) {
+        const float4 nb = nB4[c4];
+        f2_unpack(f2_add(f2_pack(__uint_as_float(rb[4 * c4]), __uint_as_float(rb[4 * c4 + 1])), f2_pack(nb.x, nb.y)), dB[0], dB[1]);
+        f2_unpack(f2_add(f2_pack(__uint_as_float(rb[4 * c4 + 2]), __uint_as_float(rb[4 * c4 + 3])), f2_pack(nb.z, nb.w)), dB[2], dB[3]);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = 4 * c4 + k;
+        float pA = ex2(dA[k]);
+        float pB = TWO ? ex2(dB[k]) : 0.f;
+        if (MASKED) {
+          const int r = s * EB_STEP + c;
+          if (r >= nR || j > a.r_lo + r) { pA = 0.f; pB = 0.f; }
+        }
+        pp[c] = f2_pack(pA, pB);
+        vs = f2_add(vs, pp[c]);
+      }
+    }
+    // transpose through the warp's buffer: row c of key l at tw[l * EB_PITCH + c]
+#pragma unroll
+    for (int c = 0; c < EB_STEP; ++c) *reinterpret_cast<uint64_t*>(&tw[l * EB_PITCH + c]) = pp[c];
+    __syncwarp();
+    // lane l sums diagonal d = c - l' + 31 = l (rows c <= l) and d = l + 32 (rows c > l)
+    uint64_t da = 0ull, db = 0ull;
+    diag_step<0, 0 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
+    diag_step<1, 1 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
+    diag_step<2, 2 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
+    diag_step<3, 3 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
+    diag_step<4, 4 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
+    diag_step<5, 5 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
+    diag_step<6, 6 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
+    diag_step<7, 7 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
+    static_assert(EB_STEP == 8, "eight diagonal steps");
+    // warp diagonal d of step s is quarter offset EB_STEP s + d (tile offset
+    // U = that + 96 - 32 q)
+    uint64_t* dsa = reinterpret_cast<uint64_t*>(&ds[s * EB_STEP + l]);
+    *dsa = f2_add(*dsa, da);
+    if (l < EB_STEP - 1) {
+      uint64_t* dsb = reinterpret_cast<uint64_t*>(&ds[s * EB_STEP + l + 32]);
+      *dsb = f2_add(*dsb, db);
+    }
+    __syncwarp();
+  }
+  return vs;
+}
+
+// Pass B epilogue warp: heads hA = 2 pi and, when TWO, hB = 2 pi + 1, key quarter q (the
+// warp's TMEM lane quarter); lane l owns key 32 q + l and keeps the two heads' values packed
+// (A, B), so one packed add, shared-memory access or exponential argument serves both.
+template <int D, bool TWO>
+__device__ __forceinline__ void est_b_epilogue(EBSmem<D>& sm, const EstArgs& a, int w, uint32_t tb,
+                                               int64_t u0, int64_t u1) {
+  const int pi = w >> 2, q = w & 3;
+  const int l = (int)lane_id();
+  const int hA = 2 * pi;
+  const int half = hA < EB_ACC0_HEADS ? 0 : 1;
+  const int bar = 1 + pi;                                   // named barrier of the pair's 4 warps
+  const uint32_t lbA = tb + ((32u * (uint32_t)q) << 16) + (uint32_t)(hA * 64);
+  float2* tw = sm.tbuf[w];
+  float2* ds = sm.dsum[pi][q];
+  // diagonal reads of row c: key l' = c + 31 - l when c <= l, else l' = c - l - 1; the
+  // element (l', c) sits at tw[l' * EB_PITCH + c], i.e. at base + c * (EB_PITCH + 1)
+  const uint32_t tw_s = smem_u32(tw);
+  const uint32_t ru = tw_s + (uint32_t)((31 - l) * EB_PITCH * 8);
+  const uint32_t rd = tw_s - (uint32_t)((l + 1) * EB_PITCH * 8);
+  const int nR = (int)(a.e - a.r_lo);
+  int g = (int)(u0 / a.nkt), kt = (int)(u0 % a.nkt);
+  int g_cur = -1;
+  bool ok = true;
+  for (int i = l; i < EB_DQ; i += 32) ds[i] = make_float2(0.f, 0.f);
+  for (int64_t u = u0, n = 0; u < u1 && ok; ++u, ++n) {
+    if (g != g_cur) {
+      // -lse of the pair's est rows, (A, B) per row (each pair keeps its own copy)
+      named_bar_sync(bar, 128);
+      {
+        const int t = 32 * q + l, hh = hA + (t >> 6), m = t & 63;
+        sm.nlse[hh][m] = hh < a.G ? -a.lse2[(int64_t)g * a.m_pad + hh * 64 + m] : 0.f;
+      }
+      named_bar_sync(bar, 128);
+      g_cur = g;
+    }
+    const bool okw = mbar_wait_sleep_warp(&sm.acc_full[half], (uint32_t)(n & 1));
+    const int64_t j = (int64_t)kt * 128 + 32 * q + l;       // this thread's key
+    if (okw) {
+      tc_fence_after();
+      // the tile reaches the estimator rows (causal mask), or the chunk has fewer rows
+      const bool masked = (int64_t)kt * 128 + 127 >= a.r_lo || nR < 64;
+      const uint64_t vs = masked ? est_b_tile<D, TWO, true>(sm, a, pi, hA, half, lbA, tw, ds, ru, rd, l, j, nR)
+                                 : est_b_tile<D, TWO, false>(sm, a, pi, hA, half, lbA, tw, ds, ru, rd, l, j, nR);
+      const int64_t hgA = (int64_t)g * a.G + hA;
+      float vA, vB;
+      f2_unpack(vs, vA, vB);
+      if (j < a.e) {
+        a.vert[hgA * a.ld + j] = vA;
+        if (TWO) a.vert[(hgA + 1) * a.ld + j] = vB;
+      }
+    }
+    // the four quarters' partials of this pair, in quarter order, into the tile's offsets
+    ok = named_bar_and(bar, 128, okw);
+    if (!ok) break;
+    const int64_t hgA = (int64_t)g * a.G + hA;
+    float* spA = a.slash_part + (hgA * a.nkt + kt) * EB_U;
+    float* spB = spA + (int64_t)a.nkt * EB_U;
+    for (int U = 32 * q + l; U < EB_U; U += 128) {
+      uint64_t acc = 0ull;
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        const int idx = U - 96 + 32 * qq;
+        if (idx >= 0 && idx < EB_DQ - 1)
+          acc = f2_add(acc, *reinterpret_cast<const uint64_t*>(&sm.dsum[pi][qq][idx]));
+      }
+      float xA, xB;
+      f2_unpack(acc, xA, xB);
+      spA[U] = xA;
+      if (TWO) spB[U] = xB;
+    }
+    named_bar_sync(bar, 128);
+    for (int i = l; i < EB_DQ; i += 32) ds[i] = make_float2(0.f, 0.f);
+    if (++kt == a.nkt) { kt = 0; ++g; }
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(EB_THREADS, 1)
@@ -226,18 +438,22 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
   extern __shared__ uint8_t eb_raw[];
   EBSmem<D>& sm = *reinterpret_cast<EBSmem<D>*>((reinterpret_cast<uintptr_t>(eb_raw) + 1023) & ~uintptr_t(1023));
   constexpr uint32_t TILE = EBSmem<D>::TILE;
+  constexpr int W_LOAD = 4 * EB_PAIRS, W_MMA = 4 * EB_PAIRS + 1;
   const int w = warp_id();
   const int Mr = a.G * 64;                                  // est rows used as N
+  const int h0 = a.G < EB_ACC0_HEADS ? a.G : EB_ACC0_HEADS;  // heads in accumulator 0
+  const int h1 = a.G - h0;                                  // heads in accumulator 1
+  const int p0 = (h0 + 1) / 2, p1 = (h1 + 1) / 2;           // head pairs per accumulator
   const int64_t W = (int64_t)a.hkv * a.nkt;
   const int64_t u0 = W * blockIdx.x / gridDim.x, u1 = W * (blockIdx.x + 1) / gridDim.x;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < EB_NK; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 1); }
+    mbar_init(&sm.k_full, 1); mbar_init(&sm.k_empty, 1);
     mbar_init(&sm.e_full, 1); mbar_init(&sm.e_empty, 1);
-    mbar_init(&sm.acc_full, 1); mbar_init(&sm.acc_free, 32 * 4 * EB_GROUPS);
+    mbar_init(&sm.acc_full[0], 1); mbar_init(&sm.acc_full[1], 1);
+    mbar_init(&sm.acc_free[0], 4 * p0); mbar_init(&sm.acc_free[1], p1 > 0 ? 4 * p1 : 1);
     mbar_init(&sm.drain, 1);
     fence_mbar_init();
   }
-  constexpr int W_LOAD = 4 * EB_GROUPS, W_MMA = 4 * EB_GROUPS + 1;
   if (w == W_MMA) { tmem_alloc(&sm.tmem_base, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -254,7 +470,7 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
         const int g = (int)(u / a.nkt), kt = (int)(u % a.nkt);
         const int key = g * 4 + est_class(a, kt);
         if (key != key_cur) {
-          ok = mbar_wait(&sm.e_empty, (en & 1) ^ 1);
+          ok = mbar_wait_sleep(&sm.e_empty, (en & 1) ^ 1);
           if (!ok) break;
           mbar_expect_tx(&sm.e_full, (uint32_t)Mr * D * 2u);
           const int cls = key & 3;
@@ -266,12 +482,11 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
           ++en;
           key_cur = key;
         }
-        const int st = (int)(n % EB_NK);
-        ok = mbar_wait(&sm.k_empty[st], ((n / EB_NK) & 1) ^ 1);
+        ok = mbar_wait_sleep(&sm.k_empty, (uint32_t)(n & 1) ^ 1u);
         if (!ok) break;
-        mbar_expect_tx(&sm.k_full[st], TILE);
+        mbar_expect_tx(&sm.k_full, TILE);
         const int y = (int)((int64_t)g * a.ld_tokens + (int64_t)kt * 128);
-        for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(sm.k[st] + hf * 16384, &mk, &sm.k_full[st], 64 * hf, y);
+        for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(sm.k + hf * 16384, &mk, &sm.k_full, 64 * hf, y);
       }
       if (!ok) { const long long c0 = clock64(); while (clock64() - c0 < 2000000) __nanosleep(1000); }
     }
@@ -279,31 +494,39 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
     if (lane_id() == 0) {
       bool ok = true;
       int key_cur = -1, en = 0;
+      // S[key][row] for est rows [r0, r0 + N) into TMEM columns [r0, r0 + N)
+      auto issue = [&](int r0, int N) {
+        const uint32_t idesc = idesc_f16(128, N, 0);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
+          const uint32_t eoff = (uint32_t)(kk >> 2) * EST_HALF + (uint32_t)r0 * 128u + (uint32_t)(kk & 3) * 32u;
+          mma_ss(tb + (uint32_t)r0, sdesc_sw128(smem_u32(sm.k) + koff, 16u, 1024u),
+                 sdesc_sw128(smem_u32(sm.est) + eoff, 16u, 1024u), idesc, kk > 0 ? 1u : 0u);
+        }
+      };
       for (int64_t u = u0, n = 0; u < u1 && ok; ++u, ++n) {
         const int g = (int)(u / a.nkt), kt = (int)(u % a.nkt);
         const int key = g * 4 + est_class(a, kt);
         if (key != key_cur) {
-          ok = mbar_wait(&sm.e_full, en & 1);
+          ok = mbar_wait_sleep(&sm.e_full, en & 1);
           if (!ok) break;
           ++en;
           key_cur = key;
         }
-        const int st = (int)(n % EB_NK);
-        ok = mbar_wait(&sm.k_full[st], (n / EB_NK) & 1) && mbar_wait(&sm.acc_free, (n & 1) ^ 1);
+        const uint32_t par = (uint32_t)(n & 1);
+        ok = mbar_wait_sleep(&sm.k_full, par) && mbar_wait_sleep(&sm.acc_free[0], par ^ 1u);
         if (!ok) break;
         tc_fence_after();
-        for (int n0 = 0; n0 < Mr; n0 += 256) {
-          const int N = Mr - n0 < 256 ? Mr - n0 : 256;
-          const uint32_t idesc = idesc_f16(128, N, 0);
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
-            const uint32_t eoff = (uint32_t)(kk >> 2) * EST_HALF + (uint32_t)n0 * 128u + (uint32_t)(kk & 3) * 32u;
-            mma_ss(tb + (uint32_t)n0, sdesc_sw128(smem_u32(sm.k[st]) + koff, 16u, 1024u),
-                   sdesc_sw128(smem_u32(sm.est) + eoff, 16u, 1024u), idesc, kk > 0 ? 1u : 0u);
-          }
+        issue(0, h0 * 64);
+        mma_commit(&sm.acc_full[0]);
+        if (h1 > 0) {
+          ok = mbar_wait_sleep(&sm.acc_free[1], par ^ 1u);
+          if (!ok) break;
+          tc_fence_after();
+          issue(h0 * 64, h1 * 64);
+          mma_commit(&sm.acc_full[1]);
         }
-        mma_commit(&sm.acc_full);
-        mma_commit(&sm.k_empty[st]);
+        mma_commit(&sm.k_empty);
         if (u + 1 >= u1) mma_commit(&sm.e_empty);
         else {
           const int64_t un = u + 1;
@@ -312,65 +535,11 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
         }
       }
       mma_commit(&sm.drain);
-      mbar_wait(&sm.drain, 0);
+      mbar_wait_sleep(&sm.drain, 0);
     }
-  } else {
-    // epilogue: group eg = w / 4 handles heads hh = eg, eg + EB_GROUPS, ...; thread owns key
-    // lane kl (its warp's TMEM lane quarter)
-    const int eg = w >> 2;
-    const int kl = 32 * (w & 3) + (int)lane_id();
-    const uint32_t lb = tb + ((32u * (w & 3)) << 16);
-    const int nR = (int)(a.e - a.r_lo);
-    int g_cur = -1;
-    bool ok = true;
-    for (int64_t u = u0, n = 0; u < u1 && ok; ++u, ++n) {
-      const int g = (int)(u / a.nkt), kt = (int)(u % a.nkt);
-      if (g != g_cur) {
-        // est rows' lse of this group (each epilogue group keeps its own copy)
-        named_bar_sync(1 + eg, 128);
-        for (int m = kl; m < Mr; m += 128) sm.lse[eg][m] = a.lse2[(int64_t)g * a.m_pad + m];
-        named_bar_sync(1 + eg, 128);
-        g_cur = g;
-      }
-      ok = named_bar_and(1 + eg, 128, mbar_wait(&sm.acc_full, n & 1));
-      if (!ok) break;
-      tc_fence_after();
-      const int64_t j = (int64_t)kt * 128 + kl;              // this thread's key
-      for (int hh = eg; hh < a.G; hh += EB_GROUPS) {
-        float vsum = 0.f;
-        float acc0 = 0.f, acc1 = 0.f;   // slash sums for U = kl and U = kl + 128
-        for (int rh = 0; rh < 64 / EB_STEP; ++rh) {
-          uint32_t rr[EB_STEP];
-          tmem_ld16(lb + (uint32_t)(hh * 64 + rh * EB_STEP), rr);
-#pragma unroll
-          for (int c = 0; c < EB_STEP; ++c) {
-            const int r = rh * EB_STEP + c;
-            const int64_t i = a.r_lo + r;
-            float p = 0.f;
-            if (r < nR && j <= i) p = ex2(__uint_as_float(rr[c]) - sm.lse[eg][hh * 64 + r]);
-            vsum += p;
-            sm.pbuf[eg][c][kl] = p;
-          }
-          named_bar_sync(1 + eg, 128);
-          // U = EB_STEP rh + c - k + 127 for row c of this step and key k of the tile
-#pragma unroll 4
-          for (int c = 0; c < EB_STEP; ++c) {
-            const int k0 = EB_STEP * rh + c + 127 - kl;
-            if (k0 >= 0 && k0 < 128) acc0 += sm.pbuf[eg][c][k0];
-            const int k1 = k0 - 128;
-            if (k1 >= 0 && k1 < 128) acc1 += sm.pbuf[eg][c][k1];
-          }
-          named_bar_sync(1 + eg, 128);
-        }
-        const int h = g * a.G + hh;
-        if (j < a.e) a.vert[(int64_t)h * a.ld + j] = vsum;
-        float* sp = a.slash_part + ((int64_t)h * a.nkt + kt) * EB_U;
-        sp[kl] = acc0;
-        if (kl + 128 < EB_U) sp[kl + 128] = acc1;
-      }
-      tc_fence_before();
-      mbar_arrive(&sm.acc_free);
-    }
+  } else if (2 * (w >> 2) < a.G) {
+    if (2 * (w >> 2) + 1 < a.G) est_b_epilogue<D, true>(sm, a, w, tb, u0, u1);
+    else est_b_epilogue<D, false>(sm, a, w, tb, u0, u1);
   }
   tc_fence_before();
   __syncthreads();
@@ -379,24 +548,18 @@ est_pass_b_kernel(const __grid_constant__ CUtensorMap me, const __grid_constant_
 }
 
 // slash[h][o] = sum of the (at most two) key tiles' partials that contain offset o, in
-// ascending tile order.
+// ascending tile order. Tile kt holds offset o at U = o - r_lo + 128 kt + 127 in [0, 190], so
+// the tiles are kt1 = floor((r_lo + 63 - o) / 128) and kt1 - 1. grid = (ceil(e / 256), hq).
 __global__ void est_slash_reduce_kernel(const EstArgs a, float* __restrict__ slash) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (int64_t)a.hq * a.e) return;
-  const int h = (int)(idx / a.e);
-  const int64_t o = idx % a.e;
-  // tile kt holds U = o - (r_lo - 128 kt - 127) in [0, 190]
-  int64_t kmin = a.r_lo - 127 - o;
-  kmin = kmin <= 0 ? 0 : (kmin + 127) / 128;
-  int64_t kmax = a.r_lo + 63 - o;
-  if (kmax < 0) { slash[(int64_t)h * a.ld + o] = 0.f; return; }
-  kmax = kmax / 128;
-  if (kmax > a.nkt - 1) kmax = a.nkt - 1;
+  const int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int h = blockIdx.y;
+  if (o >= a.e) return;
+  const int64_t kt1 = (a.r_lo + 63 - o) >> 7;               // r_lo + 63 - o >= 0 (o <= e - 1)
+  const int64_t U1 = o - a.r_lo + 128 * kt1 + 127;          // in [63, 190]
+  const float* part = a.slash_part + (int64_t)h * a.nkt * EB_U;
   float s = 0.f;
-  for (int64_t kt = kmin; kt <= kmax; ++kt) {
-    const int64_t U = o - (a.r_lo - 128 * kt - 127);
-    if (U >= 0 && U < 191) s += a.slash_part[((int64_t)h * a.nkt + kt) * EB_U + U];
-  }
+  if (kt1 >= 1 && kt1 - 1 < a.nkt && U1 >= 128) s += part[(kt1 - 1) * EB_U + (U1 - 128)];
+  if (kt1 < a.nkt && U1 < 191) s += part[kt1 * EB_U + U1];
   slash[(int64_t)h * a.ld + o] = s;
 }
 
