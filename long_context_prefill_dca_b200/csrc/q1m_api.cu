@@ -408,15 +408,17 @@ q1m_status run_rope_keys(const void* k, const void* v, int64_t s0, int64_t e, in
 
 q1m_status run_rope_queries(const void* q, int64_t s0, int64_t e, int hq, int d, const q1m_params* p,
                             const float* table, uint16_t* qv, int64_t ld_rows, cudaStream_t st) {
-  const int64_t n = ld_rows * hq * (d / 2);
   const int64_t L = p->dca_chunk - p->local_window;
   const float sc = view_scale(p, d);
   const float2* tb = reinterpret_cast<const float2*>(table);
+  // one block per row; hq * D / 16 threads of work per row
+  const int work = hq * (d / 16);
+  const int threads = work >= 256 ? 256 : (work + 31) / 32 * 32;
   if (p->in_dtype == Q1M_BF16)
-    rope_queries_kernel<__nv_bfloat16><<<blocks_for(n, 256), 256, 0, st>>>(
+    rope_queries_kernel<__nv_bfloat16><<<(unsigned)ld_rows, threads, 0, st>>>(
         (const __nv_bfloat16*)q, s0, e, hq, d, L, p->dca_chunk, sc, tb, qv, ld_rows);
   else
-    rope_queries_kernel<float><<<blocks_for(n, 256), 256, 0, st>>>(
+    rope_queries_kernel<float><<<(unsigned)ld_rows, threads, 0, st>>>(
         (const float*)q, s0, e, hq, d, L, p->dca_chunk, sc, tb, qv, ld_rows);
   Q1M_LAUNCHED();
   return Q1M_OK;
@@ -665,6 +667,8 @@ q1m_status q1m_rope_dca_queries(const void* q, int64_t s0, int64_t e, int hq, in
                                 int64_t ld_rows, void* stream) {
   Q1M_TRY(check_shape(e > 0 ? e : 1, hq, hq, d, p));
   if (!q || !table || !qv) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(table) | reinterpret_cast<uintptr_t>(qv)) & 15) != 0)
+    return fail(Q1M_ERR_INVALID, "q, table and qv must be 16-byte aligned");
   if (s0 < 0 || e <= s0 || ld_rows < e - s0 || ld_rows % 128) return fail(Q1M_ERR_INVALID, "bad row range");
   Dev dev;
   Q1M_TRY(device_info(&dev));
@@ -798,6 +802,7 @@ static q1m_status prefill_range(const void* q, const void* k, const void* v, voi
   if (first_chunk < 0 || last_chunk < first_chunk) return fail(Q1M_ERR_INVALID, "bad chunk range");
   if (!q || !k || !v || !out || !ws) return fail(Q1M_ERR_INVALID, "NULL pointer");
   if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(Q1M_ERR_INVALID, "workspace must be 256-byte aligned");
+  if (reinterpret_cast<uintptr_t>(q) & 15) return fail(Q1M_ERR_INVALID, "q must be 16-byte aligned");
   const Layout L = layout(n, hq, hkv, d, p);
   if (ws_bytes < L.total) return fail(Q1M_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   Dev dev;

@@ -83,38 +83,68 @@ __device__ __forceinline__ int64_t dca_query_pos(int64_t i, int view, int64_t L,
   return c - 1;
 }
 
+// Eight consecutive elements of one row as fp32 (16 bytes of bf16 or 32 bytes of fp32).
+__device__ __forceinline__ void load8_f32(const __nv_bfloat16* p, float* x) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    x[2 * k] = __uint_as_float(w[k] << 16);
+    x[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void load8_f32(const float* p, float* x) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
 // Query views for rows [s0, e): qv[x][h][i - s0] = scale * R(pos_x(i)) q[i][h]; rows
-// e - s0 .. ld_rows-1 are zero.
+// e - s0 .. ld_rows-1 are zero. grid.x = ld_rows (one block per row, whose three view
+// positions are then uniform); each thread rotates 8 pairs (f, f + D/2) of one head with
+// 16-byte loads and stores.
 template <typename T>
 __global__ void rope_queries_kernel(const T* __restrict__ q, int64_t s0, int64_t e, int hq,
                                     int d, int64_t L, int64_t c, float scale,
                                     const float2* __restrict__ table, uint16_t* __restrict__ qv,
                                     int64_t ld_rows) {
-  const int hd = d >> 1;
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t total = ld_rows * hq * hd;
-  if (idx >= total) return;
-  const int f = (int)(idx % hd);
-  const int h = (int)((idx / hd) % hq);
-  const int64_t r = idx / ((int64_t)hd * hq);
+  const int hd = d >> 1, n8 = hd >> 3;
+  const int64_t r = blockIdx.x;
   const int64_t i = s0 + r;
-  float x1 = 0.f, x2 = 0.f;
-  if (i < e) {
-    const int64_t src = (i * hq + h) * d;
-    x1 = load_as_f32(q + src + f) * scale;
-    x2 = load_as_f32(q + src + f + hd) * scale;
-  }
+  const bool in = i < e;
+  int64_t pos[3] = {0, 0, 0};
+  if (in) {
 #pragma unroll
-  for (int x = 0; x < 3; ++x) {
-    const int64_t dst = (((int64_t)x * hq + h) * ld_rows + r) * d;
-    uint16_t y1 = 0, y2 = 0;
-    if (i < e) {
-      const float2 cs = table[dca_query_pos(i, x, L, c) * hd + f];
-      y1 = to_f16_checked(rot_lo(x1, x2, cs));
-      y2 = to_f16_checked(rot_hi(x1, x2, cs));
+    for (int x = 0; x < 3; ++x) pos[x] = dca_query_pos(i, x, L, c);
+  }
+  for (int w = threadIdx.x; w < hq * n8; w += blockDim.x) {
+    const int h = w / n8, f0 = (w - h * n8) * 8;
+    float x1[8], x2[8];
+    if (in) {
+      const int64_t src = (i * hq + h) * d;
+      load8_f32(q + src + f0, x1);
+      load8_f32(q + src + f0 + hd, x2);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) { x1[k] *= scale; x2[k] *= scale; }
     }
-    qv[dst + f] = y1;
-    qv[dst + f + hd] = y2;
+#pragma unroll
+    for (int x = 0; x < 3; ++x) {
+      const int64_t dst = (((int64_t)x * hq + h) * ld_rows + r) * d;
+      uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
+      if (in) {
+        const float4* cs4 = reinterpret_cast<const float4*>(table + pos[x] * hd + f0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 t4 = __ldg(cs4 + k);                 // (cos, sin) of pairs 2k, 2k + 1
+          const float2 ca = make_float2(t4.x, t4.y), cb = make_float2(t4.z, t4.w);
+          lo[k] = (uint32_t)to_f16_checked(rot_lo(x1[2 * k], x2[2 * k], ca)) |
+                  ((uint32_t)to_f16_checked(rot_lo(x1[2 * k + 1], x2[2 * k + 1], cb)) << 16);
+          hi[k] = (uint32_t)to_f16_checked(rot_hi(x1[2 * k], x2[2 * k], ca)) |
+                  ((uint32_t)to_f16_checked(rot_hi(x1[2 * k + 1], x2[2 * k + 1], cb)) << 16);
+        }
+      }
+      *reinterpret_cast<uint4*>(qv + dst + f0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(qv + dst + f0 + hd) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    }
   }
 }
 
