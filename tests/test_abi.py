@@ -58,7 +58,7 @@ def test_invalid_params_rejected_without_launch(lib, field, value, code):
     p = q1m.params(C.SMALL_SPARSE)
     setattr(p, field, value)
     w = C.SMALL_SPARSE
-    st = lib.q1m_dca_sparse_prefill(1, 1, 1, 1, None, w.seq_len, w.n_q_heads, w.n_kv_heads,
+    st = lib.q1m_dca_sparse_prefill(256, 256, 256, 256, None, w.seq_len, w.n_q_heads, w.n_kv_heads,
                                     w.head_dim, ctypes.byref(p), 256, 1 << 40, None)
     assert st == code, (st, lib.q1m_last_error())
     assert lib.q1m_last_error().decode()
@@ -74,7 +74,7 @@ def test_bad_shapes_rejected(lib):
     st = lib.q1m_dca_sparse_prefill(None, 1, 1, 1, None, w.seq_len, 4, 2, 128, ctypes.byref(p),
                                     256, 1 << 40, None)
     assert st == -1
-    st = lib.q1m_dca_sparse_prefill(1, 1, 1, 1, None, w.seq_len, 4, 2, 128, ctypes.byref(p),
+    st = lib.q1m_dca_sparse_prefill(256, 256, 256, 256, None, w.seq_len, 4, 2, 128, ctypes.byref(p),
                                     256, 10, None)
     assert st == -3          # workspace too small
     # NULL device pointers: nothing here can reach a launch, whatever the order of the checks
@@ -119,7 +119,7 @@ def test_chunk_range_validated():
     lib = q1m.library()
     w = C.SMALL_SPARSE
     p = q1m.params(w)
-    args = (1, 1, 1, 1, None, w.seq_len, w.n_q_heads, w.n_kv_heads, w.head_dim, ctypes.byref(p))
+    args = (256, 256, 256, 256, None, w.seq_len, w.n_q_heads, w.n_kv_heads, w.head_dim, ctypes.byref(p))
     assert lib.q1m_dca_sparse_prefill_chunks(*args, -1, 2, 256, 1 << 40, None) == -1
     assert lib.q1m_dca_sparse_prefill_chunks(*args, 3, 2, 256, 1 << 40, None) == -1
 

@@ -82,18 +82,17 @@ def test_reference_arm_line_on_rank0():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
 
 
-def test_kernel_traffic_tracks_the_capture(tmp_path, monkeypatch):
-    """The roofline traffic figure comes from the committed ncu summary only while the
-    kernel's sources hash to the value recorded beside it, and only for its workload."""
+def test_small_case_traffic_tracks_the_capture(monkeypatch):
+    """The roofline traffic figure is the small case's capture, reported only while the
+    attention kernel's sources hash to the value recorded with it."""
     import bench
-    assert bench.kernel_traffic("7b-128k") is None
-    fake = tmp_path / "p.md"
-    fake.write_text("traffic_per_launch_bytes: 123\nkernel_source_sha256: 00\n")
-    monkeypatch.setattr(bench, "TRAFFIC_PROFILE", str(fake))
-    assert bench.kernel_traffic("7b-1m") is None
-    h = bench.kernel_source_hash()
-    fake.write_text(f"traffic_per_launch_bytes: 123\nkernel_source_sha256: {h}\n")
-    assert bench.kernel_traffic("7b-1m") == 123.0
+    monkeypatch.setitem(bench.SMALL_CASE_TRAFFIC, "bytes_per_launch", 123.0)
+    monkeypatch.setitem(bench.SMALL_CASE_TRAFFIC, "kernel_source_sha256", "00")
+    assert bench.small_case_traffic() is None
+    monkeypatch.setitem(bench.SMALL_CASE_TRAFFIC, "kernel_source_sha256", bench.kernel_source_hash())
+    assert bench.small_case_traffic() == 123.0
+    monkeypatch.setitem(bench.SMALL_CASE_TRAFFIC, "bytes_per_launch", None)
+    assert bench.small_case_traffic() is None
 
 
 def test_estimator_bounds_identities_and_ceiling():
