@@ -42,8 +42,8 @@ KERNEL_SOURCES = ("attn_tc.cuh", "q1m_device.cuh", "exp2_poly.h")
 # captured (its launches run for seconds with tens of GB resident), so its traffic is null.
 SMALL_CASE_TRAFFIC = {
     "workload": "7b-128k", "chunk": 3,
-    "bytes_per_launch": None,
-    "kernel_source_sha256": None,
+    "bytes_per_launch": 6412883000 + 1387854000,     # dram read + write, GB rounded to kB
+    "kernel_source_sha256": "69979cbce8382b1df522f55bb0cd5eb94bfeec79dbde3cb0a88a5c9dd693f556",
 }
 
 
