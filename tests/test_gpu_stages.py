@@ -105,6 +105,37 @@ def test_estimator_scores(w):
         assert np.allclose(gv.sum(1), nR, rtol=2e-3) and np.allclose(gs.sum(1), nR, rtol=2e-3)
 
 
+# every head-pair layout of the estimator's second pass: one head (a lone pair), four heads
+# (one accumulator), six and seven heads (two accumulators, the last pair full or alone); a
+# last prefill chunk of 40 rows (fewer estimator rows than 64)
+GROUPS = [
+    C.SMALL_SPARSE.with_(name=f"est-g{G}-d{D}", n_q_heads=2 * G, n_kv_heads=2, head_dim=D,
+                         seq_len=1064, prefill_chunk=512, vs_vertical=40, vs_slash=80,
+                         seed=C.SEED_BASE + 60 + G)
+    for G, D in ((1, 128), (4, 64), (6, 128), (7, 128))
+]
+
+
+@pytest.mark.parametrize("w", GROUPS, ids=lambda w: w.name)
+def test_estimator_scores_every_group_size(w):
+    x = I.generate(w)
+    g = {k: t.cuda() for k, t in x.items()}
+    orc = O.Oracle(x["q"], x["k"], x["v"], w)
+    st = Stages(w)
+    for s0, e in O.prefill_chunks(w):
+        sel = orc.select_chunk(s0, e)
+        st.keys(g["k"], g["v"], s0, e)
+        vert, slash = st.estimate(g["q"], s0, e)
+        torch.cuda.synchronize()
+        q1m.check_status()
+        gv, gs = vert.cpu().numpy(), slash.cpu().numpy()
+        nR = len(O.estimator_rows(s0, e, w))
+        for h in range(w.n_q_heads):
+            rv, rs = mean_rel(gv[h], sel.vert[h]), mean_rel(gs[h], sel.slash[h])
+            assert rv < 1e-3 and rs < 1e-3, (w.name, s0, h, rv, rs)
+            assert abs(gv[h].sum() - nR) < 2e-3 * nR and abs(gs[h].sum() - nR) < 2e-3 * nR
+
+
 def _gpu_select(w, st, vert, slash, e):
     V, S = st.select(torch.from_numpy(np.ascontiguousarray(vert)).cuda(),
                      torch.from_numpy(np.ascontiguousarray(slash)).cuda(), e)
