@@ -57,7 +57,28 @@ __device__ __forceinline__ int block_excl_scan(int v, int* tmp, int* total) {
   return res;
 }
 
-// grid (hq, 2): y = 0 vertical, y = 1 slash. One CTA selects one list of one head.
+// Order keys of scores j0 .. j0 + 3 (j0 a multiple of 4; beyond e: key 0, valid false), with
+// one 16-byte load when the row is 16-byte aligned.
+__device__ __forceinline__ void sel_keys4(const float* __restrict__ sc, int64_t j0, int64_t e, int fl,
+                                          bool vec, uint32_t (&key)[4], bool (&valid)[4]) {
+  float v[4];
+  if (vec && j0 + 3 < e) {
+    const float4 x = *reinterpret_cast<const float4*>(sc + j0);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = j0 + k < e ? sc[j0 + k] : 0.f;
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    valid[k] = j0 + k < e;
+    key[k] = valid[k] ? sel_key(v[k], j0 + k < fl) : 0u;
+  }
+}
+
+// grid (hq, 2): y = 0 vertical, y = 1 slash. One CTA selects one list of one head. Every pass
+// reads the list with 16-byte loads, several in flight per thread: the passes are bound by
+// the memory-level parallelism of one SM.
 __global__ void __launch_bounds__(SEL_THREADS)
 vs_select_kernel(const float* __restrict__ vert, const float* __restrict__ slash, int64_t ld,
                  int64_t e, int nv, int ns, int force_local, int32_t* __restrict__ V,
@@ -79,6 +100,7 @@ vs_select_kernel(const float* __restrict__ vert, const float* __restrict__ slash
     return;
   }
   if (threadIdx.x == 0) { s_prefix = 0; s_mask = 0; s_remaining = k; }
+  const bool vec = (reinterpret_cast<uintptr_t>(sc) & 15) == 0;
   const int bits[3] = {SEL_BITS0, SEL_BITS1, SEL_BITS2};
   int shift = 32;
   for (int pass = 0; pass < 3; ++pass) {
@@ -87,9 +109,17 @@ vs_select_kernel(const float* __restrict__ vert, const float* __restrict__ slash
     for (int b = threadIdx.x; b < (1 << nb); b += blockDim.x) hist[b] = 0;
     __syncthreads();
     const uint32_t pre = s_prefix, pm = s_mask;
-    for (int64_t j = threadIdx.x; j < e; j += blockDim.x) {
-      const uint32_t key = sel_key(sc[j], j < fl);
-      if ((key & pm) == pre) atomicAdd(&hist[(key >> shift) & ((1u << nb) - 1u)], 1);
+    // thread t takes elements 4 (t + i blockDim) .. + 3, four groups per iteration
+    for (int64_t base = 4 * (int64_t)threadIdx.x; base < e; base += 16 * (int64_t)blockDim.x) {
+      uint32_t key[4][4];
+      bool valid[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) sel_keys4(sc, base + 4 * (int64_t)u * blockDim.x, e, fl, vec, key[u], valid[u]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (valid[u][k] && (key[u][k] & pm) == pre) atomicAdd(&hist[(key[u][k] >> shift) & ((1u << nb) - 1u)], 1);
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -107,25 +137,63 @@ vs_select_kernel(const float* __restrict__ vert, const float* __restrict__ slash
   }
   const uint32_t T = s_prefix;
   const int need_eq = s_remaining;  // elements equal to T to take, smallest indices first
-  // ascending compaction: thread t owns the contiguous segment [t*seg, (t+1)*seg)
-  const int64_t seg = (e + blockDim.x - 1) / blockDim.x;
-  const int64_t j0 = (int64_t)threadIdx.x * seg, j1 = j0 + seg < e ? j0 + seg : e;
+  // ascending compaction: warp w owns the contiguous range [w*seg, (w+1)*seg) and reads it 128
+  // consecutive elements at a time (4 per lane); a first pass counts the keys above T and
+  // equal to T, a block scan gives each warp its output offset, a second pass writes in index
+  // order
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int64_t seg = ((e + nw - 1) / nw + 127) / 128 * 128;
+  const int64_t w0 = (int64_t)wid * seg, w1 = w0 + seg < e ? w0 + seg : e;
   int n_gt = 0, n_eq = 0;
-  for (int64_t j = j0; j < j1; ++j) {
-    const uint32_t key = sel_key(sc[j], j < fl);
-    n_gt += key > T;
-    n_eq += key == T;
+  for (int64_t base = w0; base < w1; base += 128) {
+    uint32_t key[4];
+    bool valid[4];
+    sel_keys4(sc, base + 4 * lane, w1, fl, vec, key, valid);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      n_gt += valid[k] && key[k] > T;
+      n_eq += valid[k] && key[k] == T;
+    }
   }
+  n_gt = __reduce_add_sync(0xFFFFFFFFu, (unsigned)n_gt);
+  n_eq = __reduce_add_sync(0xFFFFFFFFu, (unsigned)n_eq);
+  // warp totals -> exclusive prefix over warps (lane 0 of each warp carries the totals)
   int tot;
-  const int gt_before = block_excl_scan(n_gt, scan_tmp, &tot);
-  const int eq_before = block_excl_scan(n_eq, scan_tmp, &tot);
-  int pos = gt_before + (eq_before < need_eq ? eq_before : need_eq);
-  int eq_rank = eq_before;
-  for (int64_t j = j0; j < j1; ++j) {
-    const uint32_t key = sel_key(sc[j], j < fl);
-    if (key > T) out[pos++] = (int32_t)j;
-    else if (key == T && eq_rank < need_eq) { out[pos++] = (int32_t)j; ++eq_rank; }
-    else if (key == T) ++eq_rank;
+  const int gt_before = block_excl_scan(lane == 0 ? n_gt : 0, scan_tmp, &tot);
+  const int eq_before = block_excl_scan(lane == 0 ? n_eq : 0, scan_tmp, &tot);
+  int gt_run = __shfl_sync(0xFFFFFFFFu, gt_before, 0);   // keys above T before this step
+  int eq_run = __shfl_sync(0xFFFFFFFFu, eq_before, 0);   // keys equal to T before this step
+  for (int64_t base = w0; base < w1; base += 128) {
+    uint32_t key[4];
+    bool valid[4];
+    sel_keys4(sc, base + 4 * lane, w1, fl, vec, key, valid);
+    int c_gt = 0, c_eq = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      c_gt += valid[k] && key[k] > T;
+      c_eq += valid[k] && key[k] == T;
+    }
+    // exclusive prefix of the lanes' counts (lane order is index order)
+    int p_gt = c_gt, p_eq = c_eq;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xFFFFFFFFu, p_gt, o), b = __shfl_up_sync(0xFFFFFFFFu, p_eq, o);
+      if (lane >= o) { p_gt += a; p_eq += b; }
+    }
+    int g_before = gt_run + p_gt - c_gt, e_before = eq_run + p_eq - c_eq;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (!valid[k]) continue;
+      if (key[k] > T) {
+        out[g_before + (e_before < need_eq ? e_before : need_eq)] = (int32_t)(base + 4 * lane + k);
+        ++g_before;
+      } else if (key[k] == T) {
+        if (e_before < need_eq) out[g_before + e_before] = (int32_t)(base + 4 * lane + k);
+        ++e_before;
+      }
+    }
+    gt_run += __shfl_sync(0xFFFFFFFFu, p_gt, 31);
+    eq_run += __shfl_sync(0xFFFFFFFFu, p_eq, 31);
   }
 }
 
