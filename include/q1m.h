@@ -16,10 +16,10 @@
  * Conventions for every entry point:
  *   - Device pointers are caller-owned device memory; the library never allocates, frees or
  *     keeps them. Host pointers are named *_host.
- *   - Tensors are contiguous; q (and the query-view stage's table and qv) must be 16-byte
- *     aligned, the rotation reads and writes 16 bytes at a time. q / out are token-major
- *     [seq_len][n_q_heads][head_dim];
- *     k / v are [seq_len][n_kv_heads][head_dim]; lse is [n_q_heads][seq_len].
+ *   - Tensors are contiguous; q, k and v (and the rotation stages' table, qv, k_rot and v16)
+ *     must be 16-byte aligned: the rotations read and write 16 bytes at a time. q / out are
+ *     token-major [seq_len][n_q_heads][head_dim]; k / v are [seq_len][n_kv_heads][head_dim];
+ *     lse is [n_q_heads][seq_len].
  *   - Arguments are validated synchronously; on failure nothing is launched and a negative
  *     q1m_status is returned (q1m_last_error() gives a message). Otherwise the work is
  *     queued on `stream` (a cudaStream_t, NULL = legacy default stream) and the call returns

@@ -393,14 +393,16 @@ q1m_status run_rope_table(float* table, int64_t n_pos, int d, double base, cudaS
 q1m_status run_rope_keys(const void* k, const void* v, int64_t s0, int64_t e, int hkv, int d,
                          const q1m_params* p, const float* table, uint16_t* k_rot, uint16_t* v16,
                          int64_t ld_tokens, cudaStream_t st) {
-  const int64_t n = (e - s0) * hkv * (d / 2);
   const int64_t L = p->dca_chunk - p->local_window;
   const float2* tb = reinterpret_cast<const float2*>(table);
+  // one block per token; hkv * D / 16 threads of work per token
+  const int work = hkv * (d / 16);
+  const int threads = work >= 128 ? 128 : (work + 31) / 32 * 32;
   if (p->in_dtype == Q1M_BF16)
-    rope_keys_kernel<__nv_bfloat16><<<blocks_for(n, 256), 256, 0, st>>>(
+    rope_keys_kernel<__nv_bfloat16><<<(unsigned)(e - s0), threads, 0, st>>>(
         (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, s0, e, hkv, d, L, tb, k_rot, v16, ld_tokens);
   else
-    rope_keys_kernel<float><<<blocks_for(n, 256), 256, 0, st>>>(
+    rope_keys_kernel<float><<<(unsigned)(e - s0), threads, 0, st>>>(
         (const float*)k, (const float*)v, s0, e, hkv, d, L, tb, k_rot, v16, ld_tokens);
   Q1M_LAUNCHED();
   return Q1M_OK;
@@ -656,6 +658,9 @@ q1m_status q1m_rope_dca_keys(const void* k, const void* v, int64_t s0, int64_t e
                              int64_t ld_tokens, void* stream) {
   Q1M_TRY(check_shape(e > 0 ? e : 1, hkv, hkv, d, p));
   if (!k || !v || !table || !k_rot || !v16) return fail(Q1M_ERR_INVALID, "NULL pointer");
+  if (((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(table) |
+        reinterpret_cast<uintptr_t>(k_rot) | reinterpret_cast<uintptr_t>(v16)) & 15) != 0)
+    return fail(Q1M_ERR_INVALID, "k, v, table, k_rot and v16 must be 16-byte aligned");
   if (s0 < 0 || e <= s0 || ld_tokens < e || ld_tokens % 128) return fail(Q1M_ERR_INVALID, "bad token range");
   Dev dev;
   Q1M_TRY(device_info(&dev));
@@ -802,7 +807,8 @@ static q1m_status prefill_range(const void* q, const void* k, const void* v, voi
   if (first_chunk < 0 || last_chunk < first_chunk) return fail(Q1M_ERR_INVALID, "bad chunk range");
   if (!q || !k || !v || !out || !ws) return fail(Q1M_ERR_INVALID, "NULL pointer");
   if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(Q1M_ERR_INVALID, "workspace must be 256-byte aligned");
-  if (reinterpret_cast<uintptr_t>(q) & 15) return fail(Q1M_ERR_INVALID, "q must be 16-byte aligned");
+  if (((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15) != 0)
+    return fail(Q1M_ERR_INVALID, "q, k and v must be 16-byte aligned");
   const Layout L = layout(n, hq, hkv, d, p);
   if (ws_bytes < L.total) return fail(Q1M_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   Dev dev;

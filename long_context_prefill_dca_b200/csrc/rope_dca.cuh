@@ -53,36 +53,6 @@ __global__ void rope_table_kernel(float2* table, int64_t n_pos, int half_d, doub
   table[idx] = make_float2((float)c, (float)s);
 }
 
-// Keys [s0, e): k_rot[g][j] = R(j mod L) k[j][g]; v16[g][j] = v[j][g]; fp16.
-template <typename T>
-__global__ void rope_keys_kernel(const T* __restrict__ k, const T* __restrict__ v, int64_t s0,
-                                 int64_t e, int hkv, int d, int64_t L,
-                                 const float2* __restrict__ table, uint16_t* __restrict__ k_rot,
-                                 uint16_t* __restrict__ v16, int64_t ld_tokens) {
-  const int hd = d >> 1;
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t total = (e - s0) * hkv * hd;
-  if (idx >= total) return;
-  const int f = (int)(idx % hd);
-  const int g = (int)((idx / hd) % hkv);
-  const int64_t j = s0 + idx / ((int64_t)hd * hkv);
-  const int64_t src = (j * hkv + g) * d;
-  const float x1 = load_as_f32(k + src + f), x2 = load_as_f32(k + src + f + hd);
-  const float2 cs = table[(j % L) * hd + f];
-  const int64_t dst = ((int64_t)g * ld_tokens + j) * d;
-  k_rot[dst + f] = to_f16_checked(rot_lo(x1, x2, cs));
-  k_rot[dst + f + hd] = to_f16_checked(rot_hi(x1, x2, cs));
-  v16[dst + f] = to_f16_checked(load_as_f32(v + src + f));
-  v16[dst + f + hd] = to_f16_checked(load_as_f32(v + src + f + hd));
-}
-
-__device__ __forceinline__ int64_t dca_query_pos(int64_t i, int view, int64_t L, int64_t c) {
-  const int64_t t = i % L;
-  if (view == VIEW_INTRA) return t;
-  if (view == VIEW_SUCC) return t + L < c - 1 ? t + L : c - 1;
-  return c - 1;
-}
-
 // Eight consecutive elements of one row as fp32 (16 bytes of bf16 or 32 bytes of fp32).
 __device__ __forceinline__ void load8_f32(const __nv_bfloat16* p, float* x) {
   const uint4 u = *reinterpret_cast<const uint4*>(p);
@@ -96,6 +66,54 @@ __device__ __forceinline__ void load8_f32(const __nv_bfloat16* p, float* x) {
 __device__ __forceinline__ void load8_f32(const float* p, float* x) {
   const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
   x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+// Keys [s0, e): k_rot[g][j] = R(j mod L) k[j][g]; v16[g][j] = v[j][g]; fp16. grid.x = e - s0
+// (one block per token); each thread rotates 8 pairs (f, f + D/2) of one KV head with 16-byte
+// loads and stores, and converts the same 16 elements of v.
+template <typename T>
+__global__ void rope_keys_kernel(const T* __restrict__ k, const T* __restrict__ v, int64_t s0,
+                                 int64_t e, int hkv, int d, int64_t L,
+                                 const float2* __restrict__ table, uint16_t* __restrict__ k_rot,
+                                 uint16_t* __restrict__ v16, int64_t ld_tokens) {
+  const int hd = d >> 1, n8 = hd >> 3;
+  const int64_t j = s0 + blockIdx.x;
+  if (j >= e) return;
+  const float2* trow = table + (j % L) * hd;
+  for (int w = threadIdx.x; w < hkv * n8; w += blockDim.x) {
+    const int g = w / n8, f0 = (w - g * n8) * 8;
+    const int64_t src = (j * hkv + g) * d;
+    const int64_t dst = ((int64_t)g * ld_tokens + j) * d;
+    float x1[8], x2[8], v1[8], v2[8];
+    load8_f32(k + src + f0, x1);
+    load8_f32(k + src + f0 + hd, x2);
+    load8_f32(v + src + f0, v1);
+    load8_f32(v + src + f0 + hd, v2);
+    const float4* cs4 = reinterpret_cast<const float4*>(trow + f0);
+    uint32_t lo[4], hi[4], vl[4], vh[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 t4 = __ldg(cs4 + q);                 // (cos, sin) of pairs 2q, 2q + 1
+      const float2 ca = make_float2(t4.x, t4.y), cb = make_float2(t4.z, t4.w);
+      lo[q] = (uint32_t)to_f16_checked(rot_lo(x1[2 * q], x2[2 * q], ca)) |
+              ((uint32_t)to_f16_checked(rot_lo(x1[2 * q + 1], x2[2 * q + 1], cb)) << 16);
+      hi[q] = (uint32_t)to_f16_checked(rot_hi(x1[2 * q], x2[2 * q], ca)) |
+              ((uint32_t)to_f16_checked(rot_hi(x1[2 * q + 1], x2[2 * q + 1], cb)) << 16);
+      vl[q] = (uint32_t)to_f16_checked(v1[2 * q]) | ((uint32_t)to_f16_checked(v1[2 * q + 1]) << 16);
+      vh[q] = (uint32_t)to_f16_checked(v2[2 * q]) | ((uint32_t)to_f16_checked(v2[2 * q + 1]) << 16);
+    }
+    *reinterpret_cast<uint4*>(k_rot + dst + f0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint4*>(k_rot + dst + f0 + hd) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(v16 + dst + f0) = make_uint4(vl[0], vl[1], vl[2], vl[3]);
+    *reinterpret_cast<uint4*>(v16 + dst + f0 + hd) = make_uint4(vh[0], vh[1], vh[2], vh[3]);
+  }
+}
+
+__device__ __forceinline__ int64_t dca_query_pos(int64_t i, int view, int64_t L, int64_t c) {
+  const int64_t t = i % L;
+  if (view == VIEW_INTRA) return t;
+  if (view == VIEW_SUCC) return t + L < c - 1 ? t + L : c - 1;
+  return c - 1;
 }
 
 // Query views for rows [s0, e): qv[x][h][i - s0] = scale * R(pos_x(i)) q[i][h]; rows
