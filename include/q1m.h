@@ -48,7 +48,7 @@ extern "C" {
 typedef enum {
   Q1M_OK = 0,
   Q1M_ERR_INVALID = -1,      /* a bad argument (null pointer, bad size or shape)          */
-  Q1M_ERR_UNSUPPORTED = -2,  /* a valid case this build does not handle (head_dim, GPU)   */
+  Q1M_ERR_UNSUPPORTED = -2,  /* a valid case the library does not handle (head_dim, GPU) */
   Q1M_ERR_WORKSPACE = -3,    /* workspace too small                                        */
   Q1M_ERR_CUDA = -4,         /* a CUDA runtime call failed                                 */
   Q1M_ERR_TIMEOUT = -5,      /* a device-side bounded wait ran out (latched on the device) */
