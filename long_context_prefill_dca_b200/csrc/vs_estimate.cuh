@@ -27,7 +27,7 @@
 
 namespace q1m {
 
-constexpr int EA_THREADS = 192;   // warps 0-3 softmax, 4 loader, 5 MMA
+constexpr int EA_THREADS = 320;   // warps 0-7 softmax (two per TMEM lane quarter), 8 loader, 9 MMA
 constexpr int EA_NK = 2;
 constexpr int EB_PAIRS = 4;                            // head pairs (0,1) (2,3) (4,5) (6)
 constexpr int EB_THREADS = 32 * (4 * EB_PAIRS + 2);    // warps 0-15 epilogue, 16 loader, 17 MMA
@@ -60,20 +60,20 @@ __device__ __forceinline__ int est_class(const EstArgs& a, int kt) {
   return d >= 3 ? 3 : (int)d;
 }
 
-// One key tile of a pass A row: the online log2-sum-exp2 (mx, l) of row values x[0..127]
+// 64 keys of a pass A row: the online log2-sum-exp2 (mx, l) of row values x[0..63]
 // (log2-scaled logits). MASKED: keys c > lim are not causal for the row.
 template <bool MASKED>
-__device__ __forceinline__ void est_a_tile(float (&x)[128], int64_t lim, float& mx, float& l) {
+__device__ __forceinline__ void est_a_half(float (&x)[64], int64_t lim, float& mx, float& l) {
   if (MASKED) {
 #pragma unroll
-    for (int c = 0; c < 128; ++c) if (c > lim) x[c] = -INFINITY;
+    for (int c = 0; c < 64; ++c) if (c > lim) x[c] = -INFINITY;
   }
-  // tile maximum: eight independent chains, then a tree
+  // maximum: eight independent chains, then a tree
   float m8[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) m8[k] = x[k];
 #pragma unroll
-  for (int c = 8; c < 128; c += 8)
+  for (int c = 8; c < 64; c += 8)
 #pragma unroll
     for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], x[c + k]);
 #pragma unroll
@@ -86,7 +86,7 @@ __device__ __forceinline__ void est_a_tile(float (&x)[128], int64_t lim, float& 
   const uint64_t nmn = f2_pack(-mn, -mn);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-  for (int c = 0; c < 64; ++c) {
+  for (int c = 0; c < 32; ++c) {
     float d0, d1;
     f2_unpack(f2_add(f2_pack(x[2 * c], x[2 * c + 1]), nmn), d0, d1);
     acc[c & 3] = f2_add(acc[c & 3], f2_pack(ex2(d0), ex2(d1)));
@@ -107,6 +107,7 @@ struct EASmem {
   alignas(1024) uint8_t q[TILE];
   alignas(1024) uint8_t k[EA_NK][TILE];
   uint64_t k_full[EA_NK], k_empty[EA_NK], q_full, q_empty, s_full[2], s_free[2], drain;
+  float2 half_part[128];                  // (max, sum) of each row over the key columns 64..127
   uint32_t tmem_base;
 };
 
@@ -126,16 +127,16 @@ est_pass_a_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < EA_NK; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 1); }
     mbar_init(&sm.q_full, 1); mbar_init(&sm.q_empty, 1);
-    for (int b = 0; b < 2; ++b) { mbar_init(&sm.s_full[b], 1); mbar_init(&sm.s_free[b], 128); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&sm.s_full[b], 1); mbar_init(&sm.s_free[b], 256); }
     mbar_init(&sm.drain, 1);
     fence_mbar_init();
   }
-  if (w == 5) { tmem_alloc(&sm.tmem_base, 256); tmem_relinquish(); }
+  if (w == 9) { tmem_alloc(&sm.tmem_base, 256); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = sm.tmem_base;
-  if (w == 4) {
+  if (w == 8) {
     if (lane_id() == 0) {
       bool ok = true;
       int cls_cur = -1, qn = 0;
@@ -159,7 +160,7 @@ est_pass_a_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
       }
       if (!ok) { const long long c0 = clock64(); while (clock64() - c0 < 2000000) __nanosleep(1000); }
     }
-  } else if (w == 5) {
+  } else if (w == 9) {
     if (lane_id() == 0) {
       constexpr uint32_t IDESC = idesc_f16(128, 128, 0);
       bool ok = true;
@@ -189,13 +190,16 @@ est_pass_a_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
       mbar_wait_sleep(&sm.drain, 0);
     }
   } else {
-    // softmax: thread t owns est row m = mt * 128 + t
-    const int t = threadIdx.x;
+    // softmax: warp w takes the rows of TMEM lane quarter w & 3 (thread t owns est row
+    // m = mt * 128 + t) and the key columns [64 ch, 64 ch + 64) of each tile, ch = w >> 2; the
+    // two column halves' (max, sum) of a row are merged once at the end
+    const int ch = w >> 2;
+    const int t = threadIdx.x & 127;
     const int m = mt * 128 + t;
     const int hh = m / 64, r = m % 64;
     const int64_t i = a.r_lo + r;
     const bool live = hh < a.G && i < a.e;
-    const uint32_t lb = tb + ((32u * (warp_id() & 3u)) << 16);
+    const uint32_t lb = tb + ((32u * (warp_id() & 3u)) << 16) + 64u * (uint32_t)ch;
     float mx = -INFINITY, l = 0.f;
     bool ok = true;
     // a warp whose 32 est rows are all padding (past the group's G x 64 rows) only frees the
@@ -211,20 +215,29 @@ est_pass_a_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         mbar_arrive(&sm.s_free[b]);
         continue;
       }
-      float x[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lb + 128u * b + 32u * c, reinterpret_cast<uint32_t*>(x) + 32 * c);
+      float x[64];
+      tmem_ld64(lb + 128u * b, reinterpret_cast<uint32_t*>(x));
       tc_fence_before();
       mbar_arrive(&sm.s_free[b]);
-      if ((int64_t)kt * 128 + 127 > a.r_lo) est_a_tile<true>(x, i - (int64_t)kt * 128, mx, l);
-      else est_a_tile<false>(x, 0, mx, l);
+      const int64_t k0 = (int64_t)kt * 128 + 64 * ch;           // first key of this half
+      if (k0 + 63 > a.r_lo) est_a_half<true>(x, i - k0, mx, l);
+      else est_a_half<false>(x, 0, mx, l);
     }
-    if (ok) a.part[((int64_t)g * a.n_mt * 128 + m) * a.nsplit + split] = make_float2(live ? mx : -INFINITY, live ? l : 0.f);
+    // merge the two column halves of each row: warps 4-7 hand theirs to warps 0-3
+    if (ch == 1) sm.half_part[t] = make_float2(mx, l);
+    ok = named_bar_and(1, 256, ok);
+    if (ok && ch == 0) {
+      const float2 o = sm.half_part[t];
+      const float M = fmaxf(mx, o.x);
+      float L = 0.f;
+      if (M != -INFINITY) L = (l > 0.f ? l * ex2(mx - M) : 0.f) + (o.y > 0.f ? o.y * ex2(o.x - M) : 0.f);
+      a.part[((int64_t)g * a.n_mt * 128 + m) * a.nsplit + split] = make_float2(live ? M : -INFINITY, live ? L : 0.f);
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (w == 5) { __syncwarp(); tmem_dealloc(tb, 256); }
+  if (w == 9) { __syncwarp(); tmem_dealloc(tb, 256); }
 }
 
 // lse2[g][m] = log2 sum over splits of l * 2^max
