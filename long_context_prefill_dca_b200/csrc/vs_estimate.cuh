@@ -32,7 +32,6 @@ constexpr int EA_NK = 2;
 constexpr int EB_PAIRS = 4;                            // head pairs (0,1) (2,3) (4,5) (6)
 constexpr int EB_THREADS = 32 * (4 * EB_PAIRS + 2);    // warps 0-15 epilogue, 16 loader, 17 MMA
 constexpr int EB_STEP = 8;        // est rows per epilogue step
-constexpr int EB_PITCH = EB_STEP + 1;   // float2 per key in a warp's transpose buffer (no bank conflicts)
 constexpr int EB_ACC0_HEADS = 4;  // accumulator 0 holds heads 0..3, accumulator 1 heads 4..6
 constexpr int EB_MAX_ROWS = 448;
 constexpr int EB_U = 192;         // offsets per key tile (64 + 128 - 1 used)
@@ -268,27 +267,43 @@ struct EBSmem {
   static constexpr int EST = EB_MAX_ROWS * D * 2;
   alignas(1024) uint8_t est[EST];         // est rows, [half][row][64 halfs] swizzled
   alignas(1024) uint8_t k[TILE];          // one key tile (the epilogue covers its reload)
-  float2 tbuf[4 * EB_PAIRS][32 * EB_PITCH];  // per epilogue warp: p of 32 keys x EB_STEP rows
   float2 dsum[EB_PAIRS][4][EB_DQ];        // per head pair and key quarter: diagonal partials
   float nlse[2 * EB_PAIRS][64];           // per head and est row: -(log2-sum-exp2)
   uint64_t k_full, k_empty, e_full, e_empty, acc_full[2], acc_free[2], drain;
   uint32_t tmem_base;
 };
 
-// One element of a diagonal read: with q = (c <= l), load the packed pair at
-// (q ? ru : rd) + off and add it to da if q, else to db (predicated, no branch).
-template <int C, int OFF>
-__device__ __forceinline__ void diag_step(uint64_t& da, uint64_t& db, uint32_t ru, uint32_t rd, int l) {
+// One element of a diagonal sum: v (a packed pair of row C of another lane's key) goes into
+// da when C <= l, else into db (predicated, no branch).
+template <int C>
+__device__ __forceinline__ void diag_add(uint64_t& da, uint64_t& db, uint64_t v, int l) {
   asm volatile(
-      "{\n\t.reg .pred q;\n\t.reg .b32 ad;\n\t.reg .b64 v;\n\t"
-      "setp.le.s32 q, %4, %5;\n\t"
-      "selp.b32 ad, %2, %3, q;\n\t"
-      "ld.shared.b64 v, [ad+%6];\n\t"
-      "@q add.rn.f32x2 %0, %0, v;\n\t"
-      "@!q add.rn.f32x2 %1, %1, v;\n\t}"
+      "{\n\t.reg .pred q;\n\t"
+      "setp.le.s32 q, %3, %4;\n\t"
+      "@q add.rn.f32x2 %0, %0, %2;\n\t"
+      "@!q add.rn.f32x2 %1, %1, %2;\n\t}"
       : "+l"(da), "+l"(db)
-      : "r"(ru), "r"(rd), "n"(C), "r"(l), "n"(OFF)
-      : "memory");
+      : "l"(v), "n"(C), "r"(l));
+}
+
+// Row C of the key of lane (C - 1 - l) mod 32, fetched by a shuffle into lane l: it lies on
+// warp diagonal d = C - key + 31, which is d = l when C <= l and d = l + 32 when C > l.
+template <int C>
+__device__ __forceinline__ void diag_fetch_add(uint64_t& da, uint64_t& db, uint64_t p, int l) {
+  float x, y;
+  f2_unpack(p, x, y);
+  const int src = (C - 1 - l) & 31;
+  x = __shfl_sync(0xffffffffu, x, src);
+  y = __shfl_sync(0xffffffffu, y, src);
+  diag_add<C>(da, db, f2_pack(x, y), l);
+}
+
+template <int C>
+__device__ __forceinline__ void diag_all(uint64_t& da, uint64_t& db, const uint64_t* pp, int l) {
+  if constexpr (C < EB_STEP) {
+    diag_fetch_add<C>(da, db, pp[C], l);
+    diag_all<C + 1>(da, db, pp, l);
+  }
 }
 
 // One key tile of a pass B epilogue warp: p = 2^(s - lse) for the warp's 32 keys and its
@@ -297,14 +312,19 @@ __device__ __forceinline__ void diag_step(uint64_t& da, uint64_t& db, uint32_t r
 // not causal) or the chunk has fewer than 64 rows.
 template <int D, bool TWO, bool MASKED>
 __device__ __forceinline__ uint64_t est_b_tile(EBSmem<D>& sm, const EstArgs& a, int pi, int hA, int half,
-                                               uint32_t lbA, float2* tw, float2* ds, uint32_t ru,
-                                               uint32_t rd, int l, int64_t j, int nR) {
+                                               uint32_t lbA, float2* ds, int l, int64_t j, int nR) {
   uint64_t vs = 0ull;                                       // vertical sums (A, B)
 #pragma unroll 1
   for (int s = 0; s < 64 / EB_STEP; ++s) {
     uint32_t ra[EB_STEP], rb[EB_STEP];
-    tmem_ld8(lbA + (uint32_t)(s * EB_STEP), ra);
-    if (TWO) tmem_ld8(lbA + 64u + (uint32_t)(s * EB_STEP), rb);
+    static_assert(EB_STEP == 8 || EB_STEP == 16, "one TMEM load per head and step");
+    if constexpr (EB_STEP == 8) {
+      tmem_ld8(lbA + (uint32_t)(s * EB_STEP), ra);
+      if (TWO) tmem_ld8(lbA + 64u + (uint32_t)(s * EB_STEP), rb);
+    } else {
+      tmem_ld16(lbA + (uint32_t)(s * EB_STEP), ra);
+      if (TWO) tmem_ld16(lbA + 64u + (uint32_t)(s * EB_STEP), rb);
+    }
     if (s == 64 / EB_STEP - 1) {
       // every TMEM read of this tile is done: the MMA may overwrite the accumulator
       tc_fence_before();
@@ -340,21 +360,10 @@ __device__ __forceinline__ uint64_t est_b_tile(EBSmem<D>& sm, const EstArgs& a, 
         vs = f2_add(vs, pp[c]);
       }
     }
-    // transpose through the warp's buffer: row c of key l at tw[l * EB_PITCH + c]
-#pragma unroll
-    for (int c = 0; c < EB_STEP; ++c) *reinterpret_cast<uint64_t*>(&tw[l * EB_PITCH + c]) = pp[c];
-    __syncwarp();
-    // lane l sums diagonal d = c - l' + 31 = l (rows c <= l) and d = l + 32 (rows c > l)
+    // diagonal sums across the warp's 32 keys: lane l sums warp diagonal l (rows c <= l)
+    // and l + 32 (rows c > l), rows in ascending order
     uint64_t da = 0ull, db = 0ull;
-    diag_step<0, 0 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
-    diag_step<1, 1 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
-    diag_step<2, 2 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
-    diag_step<3, 3 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
-    diag_step<4, 4 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
-    diag_step<5, 5 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
-    diag_step<6, 6 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
-    diag_step<7, 7 * (EB_PITCH + 1) * 8>(da, db, ru, rd, l);
-    static_assert(EB_STEP == 8, "eight diagonal steps");
+    diag_all<0>(da, db, pp, l);
     // warp diagonal d of step s is quarter offset EB_STEP s + d (tile offset
     // U = that + 96 - 32 q)
     uint64_t* dsa = reinterpret_cast<uint64_t*>(&ds[s * EB_STEP + l]);
@@ -380,13 +389,7 @@ __device__ __forceinline__ void est_b_epilogue(EBSmem<D>& sm, const EstArgs& a, 
   const int half = hA < EB_ACC0_HEADS ? 0 : 1;
   const int bar = 1 + pi;                                   // named barrier of the pair's 4 warps
   const uint32_t lbA = tb + ((32u * (uint32_t)q) << 16) + (uint32_t)(hA * 64);
-  float2* tw = sm.tbuf[w];
   float2* ds = sm.dsum[pi][q];
-  // diagonal reads of row c: key l' = c + 31 - l when c <= l, else l' = c - l - 1; the
-  // element (l', c) sits at tw[l' * EB_PITCH + c], i.e. at base + c * (EB_PITCH + 1)
-  const uint32_t tw_s = smem_u32(tw);
-  const uint32_t ru = tw_s + (uint32_t)((31 - l) * EB_PITCH * 8);
-  const uint32_t rd = tw_s - (uint32_t)((l + 1) * EB_PITCH * 8);
   const int nR = (int)(a.e - a.r_lo);
   int g = (int)(u0 / a.nkt), kt = (int)(u0 % a.nkt);
   int g_cur = -1;
@@ -409,8 +412,8 @@ __device__ __forceinline__ void est_b_epilogue(EBSmem<D>& sm, const EstArgs& a, 
       tc_fence_after();
       // the tile reaches the estimator rows (causal mask), or the chunk has fewer rows
       const bool masked = (int64_t)kt * 128 + 127 >= a.r_lo || nR < 64;
-      const uint64_t vs = masked ? est_b_tile<D, TWO, true>(sm, a, pi, hA, half, lbA, tw, ds, ru, rd, l, j, nR)
-                                 : est_b_tile<D, TWO, false>(sm, a, pi, hA, half, lbA, tw, ds, ru, rd, l, j, nR);
+      const uint64_t vs = masked ? est_b_tile<D, TWO, true>(sm, a, pi, hA, half, lbA, ds, l, j, nR)
+                                 : est_b_tile<D, TWO, false>(sm, a, pi, hA, half, lbA, ds, l, j, nR);
       const int64_t hgA = (int64_t)g * a.G + hA;
       float vA, vB;
       f2_unpack(vs, vA, vB);
