@@ -59,13 +59,39 @@ __device__ __forceinline__ int est_class(const EstArgs& a, int kt) {
   return d >= 3 ? 3 : (int)d;
 }
 
-// 64 keys of a pass A row: the online log2-sum-exp2 (mx, l) of row values x[0..63]
-// (log2-scaled logits). MASKED: keys c > lim are not causal for the row.
+// 64 keys of a pass A row: the log2-sum-exp2 of row values x[0..63] (log2-scaled logits)
+// added into (mx, l), which stands for l * 2^mx. MASKED: keys c > lim are not causal for the
+// row.
+//
+// The sums are fp32, so the reference mx need not be the running maximum: any mx with every
+// 2^(x - mx) in range gives the same l * 2^mx up to rounding. The values are therefore
+// exponentiated against the current mx first. The tile is redone against its own maximum
+// only when that sum is infinite, NaN or above 2^64: on a row's first tile, where mx = -inf,
+// or when values lie far above mx. A row's accumulated l then stays below 2^77, far inside
+// fp32.
 template <bool MASKED>
 __device__ __forceinline__ void est_a_half(float (&x)[64], int64_t lim, float& mx, float& l) {
   if (MASKED) {
 #pragma unroll
     for (int c = 0; c < 64; ++c) if (c > lim) x[c] = -INFINITY;
+  }
+  if (mx != -INFINITY) {
+    const uint64_t nm = f2_pack(-mx, -mx);
+    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      float d0, d1;
+      f2_unpack(f2_add(f2_pack(x[2 * c], x[2 * c + 1]), nm), d0, d1);
+      acc[c & 3] = f2_add(acc[c & 3], f2_pack(ex2(d0), ex2(d1)));
+    }
+    float s0, s1, s2, s3;
+    f2_unpack(f2_add(acc[0], acc[1]), s0, s1);
+    f2_unpack(f2_add(acc[2], acc[3]), s2, s3);
+    const float sum = (s0 + s1) + (s2 + s3);
+    if (sum <= 0x1p64f) {                                    // false for +inf and NaN
+      l += sum;
+      return;
+    }
   }
   // maximum: eight independent chains, then a tree
   float m8[8];

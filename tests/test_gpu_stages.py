@@ -136,6 +136,54 @@ def test_estimator_scores_every_group_size(w):
             assert abs(gv[h].sum() - nR) < 2e-3 * nR and abs(gs[h].sum() - nR) < 2e-3 * nR
 
 
+# the 7B head shape (7 Q heads per KV head) on 12,288 tokens: the last prefill chunk's 96 key
+# tiles fall into 18 splits of 6 tiles in the estimator's first pass
+DOMINANT = C.SMALL_SPARSE.with_(name="est-dominant-key", seq_len=12288, n_q_heads=28, n_kv_heads=4,
+                                head_dim=128, rope_base=1e6, dca_chunk=4096, local_window=512,
+                                yarn_s=4.0, prefill_chunk=4096, vs_vertical=200, vs_slash=400,
+                                sinks=0, bands=0, seed=C.SEED_BASE + 70)
+
+
+def test_estimator_scores_with_a_dominant_late_key():
+    """One key per KV head whose logit lies 35 to 180 log2 units (depending on the row) above
+    every other key of the estimator rows. At the last prefill chunk it is in the fifth key tile
+    of its split (tile 40; splits of 6 tiles). Against the reference that a split's first tile
+    set, the rows with the larger gaps sum past 2^64 or overflow there and redo the tile against
+    its own maximum; the others keep the reference with sums up to 2^64. At the middle chunk the
+    key falls in the first tile of its split. The scores must still match the oracle and sum to
+    one per row. The planted direction is the lowest-frequency rotary pair (dimensions 63 and
+    127), which the rotations barely turn at these distances."""
+    w = DOMINANT
+    x = I.generate(w)
+    D, G = w.head_dim, w.group
+    u = np.zeros(D, np.float32)
+    u[D // 2 - 1] = u[D - 1] = np.float32(1 / np.sqrt(2))
+    pos = 40 * 128 + 37
+    q, k = x["q"].float(), x["k"].float()
+    for g in range(w.n_kv_heads):
+        q[:, g * G:(g + 1) * G, :] += 4.0 * torch.from_numpy(u)
+        k[pos, g, :] += 175.0 * torch.from_numpy(u)
+    x["q"], x["k"] = q.to(x["q"].dtype), k.to(x["k"].dtype)
+    g = {n: t.cuda() for n, t in x.items()}
+    orc = O.Oracle(x["q"], x["k"], x["v"], w)
+    st = Stages(w)
+    for s0, e in O.prefill_chunks(w):
+        sel = orc.select_chunk(s0, e)
+        st.keys(g["k"], g["v"], s0, e)
+        vert, slash = st.estimate(g["q"], s0, e)
+        torch.cuda.synchronize()
+        q1m.check_status()
+        gv, gs = vert.cpu().numpy(), slash.cpu().numpy()
+        nR = len(O.estimator_rows(s0, e, w))
+        if e > pos + 1:
+            # the planted key takes nearly all of every estimator row's probability
+            assert np.all(sel.vert[:, pos] > 0.99 * nR)
+        for h in range(w.n_q_heads):
+            rv, rs = mean_rel(gv[h], sel.vert[h]), mean_rel(gs[h], sel.slash[h])
+            assert rv < 1e-3 and rs < 1e-3, (s0, h, rv, rs)
+            assert abs(gv[h].sum() - nR) < 2e-3 * nR and abs(gs[h].sum() - nR) < 2e-3 * nR
+
+
 def _gpu_select(w, st, vert, slash, e):
     V, S = st.select(torch.from_numpy(np.ascontiguousarray(vert)).cuda(),
                      torch.from_numpy(np.ascontiguousarray(slash)).cuda(), e)
