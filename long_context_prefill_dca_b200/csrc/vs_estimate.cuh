@@ -9,18 +9,19 @@
 // The G Q heads of a KV group share keys, so the G * |R| (<= 448) estimator rows of a group
 // form one operand ("est rows", m = hh * 64 + r). Each key block picks the rows' query view
 // by its DCA chunk class (see est_queries_kernel).
-//  pass A: rows as M (128 rows per tile), keys as N; online max/sum per row over a range of
-//          key tiles; partial (max, sum) per split, merged into the row's log2-sum-exp2.
+//  pass A: rows as M (128 rows per tile), keys as N; per row a sum l of 2^(x - m) against a
+//          reference m kept from the row's first tile, over a range of key tiles; partial
+//          (m, l) per split, merged into the row's log2-sum-exp2.
 //  pass B: keys as M (128 keys per tile), est rows as N (<= 448 TMEM columns, in two
 //          accumulators: heads 0..3 and heads 4..6, so the MMA of one overlaps the epilogue
 //          of the other). One epilogue warp per (pair of heads, 32-key quarter), the two
-//          heads' values packed in float2 so that every add, shared-memory access and
-//          exponential argument serves both; each thread owns one key, so its vertical
-//          scores are thread-local sums over rows. Slash sums are sums along diagonals: each
-//          warp transposes its 32 keys x 8 rows of p through its own shared-memory buffer
-//          and sums the 39 diagonals they touch; the four quarters' diagonal partials are
-//          added per tile (192 offsets) and the two tiles that touch each offset are summed
-//          later, always in the same order, so the scores are deterministic.
+//          heads' values packed in float2 so that every add, shuffle and exponential
+//          argument serves both; each thread owns one key, so its vertical scores are
+//          thread-local sums over rows. Slash sums are sums along diagonals: for each group of
+//          8 rows, every lane fetches by warp shuffles the values of its two diagonals from
+//          the warp's 32 keys and sums them; the four quarters' diagonal partials are added
+//          per tile (192 offsets) and the two tiles that touch each offset are summed later,
+//          always in the same order, so the scores are deterministic.
 #pragma once
 
 #include "q1m_device.cuh"
@@ -343,14 +344,9 @@ __device__ __forceinline__ uint64_t est_b_tile(EBSmem<D>& sm, const EstArgs& a, 
 #pragma unroll 1
   for (int s = 0; s < 64 / EB_STEP; ++s) {
     uint32_t ra[EB_STEP], rb[EB_STEP];
-    static_assert(EB_STEP == 8 || EB_STEP == 16, "one TMEM load per head and step");
-    if constexpr (EB_STEP == 8) {
-      tmem_ld8(lbA + (uint32_t)(s * EB_STEP), ra);
-      if (TWO) tmem_ld8(lbA + 64u + (uint32_t)(s * EB_STEP), rb);
-    } else {
-      tmem_ld16(lbA + (uint32_t)(s * EB_STEP), ra);
-      if (TWO) tmem_ld16(lbA + 64u + (uint32_t)(s * EB_STEP), rb);
-    }
+    static_assert(EB_STEP == 8, "one 8-column TMEM load per head and step");
+    tmem_ld8(lbA + (uint32_t)(s * EB_STEP), ra);
+    if (TWO) tmem_ld8(lbA + 64u + (uint32_t)(s * EB_STEP), rb);
     if (s == 64 / EB_STEP - 1) {
       // every TMEM read of this tile is done: the MMA may overwrite the accumulator
       tc_fence_before();
@@ -358,7 +354,7 @@ __device__ __forceinline__ uint64_t est_b_tile(EBSmem<D>& sm, const EstArgs& a, 
       if (l == 0) mbar_arrive(&sm.acc_free[half]);
     }
     // row pairs (c, c + 1) of one head are adjacent registers: packed adds on them, then
-    // each exponential's result is paired with the other head's for the transpose
+    // each exponential's result is paired with the other head's for the shuffles
     const float4* nA4 = reinterpret_cast<const float4*>(&sm.nlse[hA][s * EB_STEP]);
     const float4* nB4 = reinterpret_cast<const float4*>(&sm.nlse[hA + 1][s * EB_STEP]);
     uint64_t pp[EB_STEP];
